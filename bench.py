@@ -1,0 +1,333 @@
+"""Benchmark: one exact Lloyd iteration (assignment + sort-inverse update) per step.
+
+Workload (the one the headline metric is quoted on): B=32 independent problems, N=65536 points
+each, d=128, K=1024 centroids, fp16 points, fp32 centroids; 1024-component Gaussian mixture per
+batch (means N(0,1)^128, sigma=0.3), init = K seeded-random points. Inputs (X = 537 MB) are
+larger than the 126 MB L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+A step on the GPU = km_assign (tensor-core FlashAssign with inertia) + km_update (histogram,
+scan, scatter, segmented reduce, finalize) + km_prep (cast of the new centroids for the next
+assignment): exactly one iteration of km_fit's loop. Multi-GPU: one process per GPU (torchrun),
+each rank runs its own B=32 workload (independent problems, no data-path collective, weak
+scaling); the step time is the max over ranks.
+
+`--impl reference` times the fp64 CPU oracle on this host (a bounded sample of the same
+workload, scaled to the full iteration) and prints the same JSON line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Lloyd iter/s & assign pt·K/s (B=32,N=65536,K=1024,d=128); % roofline"
+B, N, K, D = 32, 65536, 1024, 128
+WORKLOAD = "batched_assign_bound: B=32 N=65536 d=128 K=1024 fp16, per-batch 1024-comp GMM sigma=0.3"
+ASSIGN_FLOP = 2.0 * B * N * K * D                       # <x,c> contraction per iteration
+# algorithmic bytes of the update: X gathered once + ids read twice + perm written and read
+UPDATE_BYTES = B * N * D * 2 + 4 * B * N * 4 + B * K * D * 4 * 2
+ASSIGN_BYTES = B * N * D * 2 + B * K * D * 2 + B * N * 4
+LAUNCHES_PER_STEP = 8   # cnpad, assign_tc, hist, scan, scatter, segreduce, finalize, prep
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["bf16_tflops"]), float(j["hbm_gbs"]), "measured"
+    return 1590.0, 6650.0, "fallback"
+
+
+def _kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("km_assign_tc.cuh", "km_common.cuh"):
+        with open(os.path.join(ROOT, "exact_lloyd_means_assign_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _profile_traffic():
+    """DRAM bytes per assign launch from the committed ncu summary, if it matches this source."""
+    p = os.path.join(ROOT, "profiles", "assign_tc_batched_assign_bound.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    s = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
+    if not m or not s or s.group(1) != _kernel_source_hash():
+        return None
+    return float(m.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        rows = []
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), float(f[3]), f[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v.lower() == "active"})
+        sm = sorted(r[0] for r in rows)
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(r[2] for r in rows)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def run_gpu(args):
+    import exact_lloyd_means_assign_b200 as km
+    import synth
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+    # each rank owns its own B=32 problems (independent batches)
+    d = synth.make_workload(3, device=dev, seed=1234 + 3 + 1000 * rank)
+    X, C = d["X"], d["C0"]
+    ws_a = km.workspace(km.KM_OP_ASSIGN, B, N, K, D, X.dtype, dev)
+    ws_u = km.workspace(km.KM_OP_UPDATE, B, N, K, D, X.dtype, dev)
+    ids = torch.empty((B, N), dtype=torch.int32, device=dev)
+    counts = torch.empty((B, K), dtype=torch.int32, device=dev)
+    inertia = torch.empty((B,), dtype=torch.float64, device=dev)
+    Cx, cn = km.km_prep(C, X.dtype)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        km.km_assign(X, Cx, cn, ids=ids, inertia=inertia, ws=ws_a, stream=stream)
+        km.km_update(X, ids, C, C_new=C, counts=counts, ws=ws_u, stream=stream)
+        km.km_prep(C, X.dtype, Cx=Cx, cn=cn, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as cs:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            e = ev[i]
+            e[0].record(stream)
+            km.km_assign(X, Cx, cn, ids=ids, inertia=inertia, ws=ws_a, stream=stream)
+            e[1].record(stream)
+            km.km_update(X, ids, C, C_new=C, counts=counts, ws=ws_u, stream=stream)
+            km.km_prep(C, X.dtype, Cx=Cx, cn=cn, stream=stream)
+            e[2].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    total_ms = t0.elapsed_time(t1)
+    assign_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    update_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    vals = torch.tensor([total_ms, assign_ms, update_ms], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(vals, op=pg.ReduceOp.MAX)
+    total_ms, assign_ms, update_ms = vals.tolist()
+    ms_per_step = total_ms / args.steps
+    err = km.km_device_error()
+
+    # end to end through the public host-buffer entry point: H2D of X and C, one iteration,
+    # D2H of the new centroids and the inertia, synchronised, every step
+    Xh = X.cpu().pin_memory()
+    Ch = d["C0"].cpu().pin_memory()
+    inh = torch.empty((1, B), dtype=torch.float64).pin_memory()
+    ws_h = km.workspace(km.KM_OP_FIT_HOST, B, N, K, D, X.dtype, dev, False, 1)
+    e2e_steps = max(3, min(20, args.steps // 25))
+    km.km_fit_host(Xh, Ch, 1, inertia_host=inh, ws=ws_h, device=dev)
+    if pg:
+        pg.barrier()
+    t = time.perf_counter()
+    for _ in range(e2e_steps):
+        km.km_fit_host(Xh, Ch, 1, inertia_host=inh, ws=ws_h, device=dev)
+    e2e_s = torch.tensor([(time.perf_counter() - t) / e2e_steps], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(e2e_s, op=pg.ReduceOp.MAX)
+    e2e_s = float(e2e_s.item())
+
+    clocks = cs.summary()
+    if rank == 0:
+        peak_tf, peak_bw, peak_kind = _peaks()
+        achieved_tf = ASSIGN_FLOP / (assign_ms * 1e-3) / 1e12
+        upd_gbs = UPDATE_BYTES / (update_ms * 1e-3) / 1e9
+        traffic = _profile_traffic()
+        line = {
+            "metric": METRIC,
+            "value": ws * 1e3 / ms_per_step,
+            "unit": "iter/s",
+            "n_gpus": ws,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_per_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": B, "N": N, "K": K, "d": D, "iterations_per_step": 1,
+                       "init": "K seeded-random points per batch", "l2": "inputs larger than L2 (X = 537 MB)",
+                       "parallelism": f"batch-sharded x{ws} (independent problems, no collective)"},
+            "assign_pt_k_per_s": ws * B * N * K / (assign_ms * 1e-3),
+            "assign_ms": assign_ms,
+            "update_ms": update_ms,
+            "roofline": {"bound": "tensor", "kernel": "assign_tc_kernel (+ norm padding)",
+                         "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": achieved_tf / peak_tf, "traffic": traffic,
+                         "peak_source": f"{peak_kind} bf16 dense (fp16 nominal ratio 1.0)"},
+            "update_roofline": {"bound": "hbm", "achieved": upd_gbs, "peak": peak_bw, "unit": "GB/s",
+                                "frac": upd_gbs / peak_bw, "algorithmic_bytes": UPDATE_BYTES,
+                                "peak_source": peak_kind},
+            "e2e": {"value": ws / e2e_s, "unit": "iter/s",
+                    "h2d_bytes_per_step": B * N * D * 2 + B * K * D * 4,
+                    "d2h_bytes_per_step": B * K * D * 4 + B * 8},
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "clocks": clocks,
+            "device_error": err,
+        }
+        if ws == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(X, d["C0"], budget_s=args.cpu_budget)
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def cpu_baseline(X, C, budget_s=15.0):
+    """The fp64 oracle on a bounded sample of the workload, scaled to one full iteration."""
+    import numpy as np
+    import oracle
+    b = 0
+    Xb = oracle.as_f64(X[b:b + 1].cpu())
+    Cb = oracle.round_to_dtype(C[b:b + 1].cpu(), X.dtype)
+    n = 1024
+    t = time.perf_counter()
+    oracle.assign(Xb[:, :n], Cb)
+    per_pt = (time.perf_counter() - t) / n
+    n = int(min(N, max(1024, budget_s * 0.8 / max(per_pt, 1e-9))))
+    t = time.perf_counter()
+    ids, _, _, _ = oracle.assign(Xb[:, :n], Cb)
+    t_assign = time.perf_counter() - t
+    t = time.perf_counter()
+    oracle.update(Xb[:, :n], ids, Cb)
+    t_update = time.perf_counter() - t
+    full = (t_assign + t_update) * (B * N) / n
+    return {"value": 1.0 / full, "unit": "iter/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{n} points of batch 0 (assign + update, fp64), scaled by {B * N / n:.1f} to one "
+                      f"full iteration", "seconds_measured": t_assign + t_update}
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return
+    import oracle
+    import synth
+    d = synth.make_workload(3, B=1, N=N, device="cpu")
+    X, C = d["X"], d["C0"]
+    # a step = one bounded sample (assign + update) scaled to the full iteration
+    per_step_budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(X, C, budget_s=per_step_budget)
+    vals = []
+    last = None
+    for _ in range(args.steps):
+        last = cpu_baseline(X, C, budget_s=per_step_budget)
+        vals.append(1.0 / last["value"])
+    s_per_iter = sum(vals) / len(vals)
+    line = {
+        "metric": METRIC, "impl": "reference", "value": 1.0 / s_per_iter, "unit": "iter/s",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": s_per_iter * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": B, "N": N, "K": K, "d": D, "iterations_per_step": 1},
+        "cpu_baseline": {"value": 1.0 / s_per_iter, "unit": "iter/s", "cores": last["cores"],
+                         "kind": "oracle", "sample": last["sample"]},
+        "e2e": {"value": 1.0 / s_per_iter, "unit": "iter/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,89 @@
+// km_centroids.cuh -- per-centroid kernels: preparation for the assignment and the final divide.
+//
+// prep:     Cx = C rounded to the points' dtype, cn = ||Cx||^2 (fp32), one warp per centroid.
+// finalize: C_new = sums / wsum for non-empty clusters, else C_prev (the mean S_j / N_j of the
+//           Lloyd recap in the steinslab e-means daily); optionally also Cx and cn for the next
+//           assignment, so a multi-iteration fit never runs prep twice.
+// cnpad:    the norm row the tensor-core assignment reads, padded to whole centroid tiles with
+//           +inf so padding columns can never win the argmin.
+#pragma once
+
+#include "km_common.cuh"
+
+namespace km {
+
+template <typename T>
+__global__ void prep_kernel(const float *__restrict__ C, int64_t rows, int d, T *__restrict__ Cx,
+                            float *__restrict__ cn) {
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const float *c = C + row * d;
+    float s = 0.f;
+    for (int j = lane; j < d; j += 32) {
+        const T v = Cvt<T>::from_f(c[j]);
+        if (Cx) Cx[row * d + j] = v;
+        const float f = Cvt<T>::to_f(v);
+        s = fmaf(f, f, s);
+    }
+    s = warp_sum(s);
+    if (lane == 0 && cn) cn[row] = s;
+}
+
+// C_prev and C_new may alias (each element is read and then written by the same thread).
+template <typename T>
+__global__ void finalize_kernel(const float *__restrict__ sums, const float *__restrict__ wsum,
+                                const int32_t *__restrict__ counts, const float *C_prev,
+                                int64_t rows, int d, float *C_new, T *__restrict__ Cx,
+                                float *__restrict__ cn) {
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const int cnt = counts[row];
+    const float div = wsum ? wsum[row] : static_cast<float>(cnt);
+    const bool upd = cnt > 0 && div > 0.f;
+    float s = 0.f;
+    for (int j = lane; j < d; j += 32) {
+        const int64_t e = row * d + j;
+        const float v = upd ? sums[e] / div : C_prev[e];
+        C_new[e] = v;
+        if (Cx) {
+            const T t = Cvt<T>::from_f(v);
+            Cx[e] = t;
+            const float f = Cvt<T>::to_f(t);
+            s = fmaf(f, f, s);
+        }
+    }
+    if (cn) {
+        s = warp_sum(s);
+        if (lane == 0) cn[row] = s;
+    }
+}
+
+// cnp[b, k] for k < Kp: ||Cx[b,k]||^2 (from `cn` when given, else computed from Cx) for k < K,
+// +inf for the padding k >= K. One warp per (b, k).
+template <typename T>
+__global__ void cnpad_kernel(const T *__restrict__ Cx, const float *__restrict__ cn, int B, int K,
+                             int Kp, int d, float *__restrict__ cnp) {
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= static_cast<int64_t>(B) * Kp) return;
+    const int b = static_cast<int>(row / Kp), k = static_cast<int>(row % Kp);
+    float v;
+    if (k >= K) {
+        v = INFINITY;
+    } else if (cn) {
+        v = cn[static_cast<int64_t>(b) * K + k];
+    } else {
+        const T *c = Cx + (static_cast<int64_t>(b) * K + k) * d;
+        float s = 0.f;
+        for (int j = lane; j < d; j += 32) {
+            const float f = Cvt<T>::to_f(c[j]);
+            s = fmaf(f, f, s);
+        }
+        v = warp_sum(s);
+    }
+    if (lane == 0) cnp[row] = v;
+}
+
+}  // namespace km

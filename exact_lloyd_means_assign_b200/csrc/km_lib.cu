@@ -1,0 +1,644 @@
+// km_lib.cu -- the C ABI of libkmeans_b200.so (declared in include/kmeans_b200.h).
+//
+// Argument validation, workspace carving, kernel selection and stream-ordered launches. All
+// kernels live in the km_*.cuh headers of this directory and are compiled in this single
+// translation unit. The library never allocates device memory: every scratch buffer is carved
+// from the caller's workspace, whose size km_workspace_size computes with the same layout code.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+
+#include "kmeans_b200.h"
+#include "km_assign_simt.cuh"
+#include "km_assign_tc.cuh"
+#include "km_centroids.cuh"
+#include "km_common.cuh"
+#include "km_fit1d.cuh"
+#include "km_update.cuh"
+
+namespace {
+
+using km::Cvt;
+
+constexpr size_t kAlign = 256;
+constexpr int64_t kMaxIndex = (int64_t{1} << 31) - 1;
+constexpr int64_t kMaxD = int64_t{1} << 20;
+constexpr int kMaxGridY = 65535;
+
+inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline cudaStream_t S(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool valid_dtype(km_dtype dt) { return dt == KM_F32 || dt == KM_F16 || dt == KM_BF16; }
+inline size_t dtype_size(km_dtype dt) { return dt == KM_F32 ? 4 : 2; }
+
+inline bool sizes_ok(int64_t B, int64_t N, int64_t K, int64_t d) {
+    return B >= 1 && N >= 1 && K >= 1 && d >= 1 && B <= kMaxIndex && N <= kMaxIndex &&
+           K <= kMaxIndex && d <= kMaxD && B * N <= (int64_t{1} << 40) &&
+           B * K <= (int64_t{1} << 40);
+}
+
+// ---------------------------------------------------------------- workspace layouts
+
+struct Carver {
+    uint8_t *base;
+    size_t off = 0;
+    explicit Carver(void *b) : base(static_cast<uint8_t *>(b)) {}
+    template <typename P> P *take(size_t bytes) {
+        P *p = base ? reinterpret_cast<P *>(base + off) : nullptr;
+        off += align_up(bytes);
+        return p;
+    }
+};
+
+inline bool tc_shape_ok(km_dtype dt, int64_t d) {
+    return dt != KM_F32 && d % 8 == 0 && d >= 8 && d <= 256;
+}
+inline int tc_bn(int64_t K) { return K > 128 ? 256 : (K > 64 ? 128 : 64); }
+inline int64_t tc_kp(int64_t K) { return ceil_div(K, tc_bn(K)) * tc_bn(K); }
+
+inline size_t ws_assign(int64_t B, int64_t K, int64_t d, km_dtype dt) {
+    return tc_shape_ok(dt, d) ? align_up(static_cast<size_t>(B * tc_kp(K)) * 4) : 0;
+}
+
+struct UpdateWs {
+    int32_t *offsets, *cursor, *perm;
+    float *sums, *wsum;
+};
+inline UpdateWs carve_update(Carver &c, int64_t B, int64_t N, int64_t K, int64_t d) {
+    UpdateWs u;
+    u.offsets = c.take<int32_t>(static_cast<size_t>(B * (K + 1)) * 4);
+    u.cursor = c.take<int32_t>(static_cast<size_t>(B * K) * 4);
+    u.perm = c.take<int32_t>(static_cast<size_t>(B * N) * 4);
+    u.sums = c.take<float>(static_cast<size_t>(B * K * d) * 4);
+    u.wsum = c.take<float>(static_cast<size_t>(B * K) * 4);
+    return u;
+}
+
+struct FitWs {
+    void *Cx;
+    float *cn;
+    int32_t *ids, *counts;
+    double *inertia;
+    void *rest;
+};
+inline FitWs carve_fit(Carver &c, int64_t B, int64_t N, int64_t K, int64_t d, km_dtype dt) {
+    FitWs f;
+    f.Cx = c.take<uint8_t>(static_cast<size_t>(B * K * d) * dtype_size(dt));
+    f.cn = c.take<float>(static_cast<size_t>(B * K) * 4);
+    f.ids = c.take<int32_t>(static_cast<size_t>(B * N) * 4);
+    f.counts = c.take<int32_t>(static_cast<size_t>(B * K) * 4);
+    f.inertia = c.take<double>(static_cast<size_t>(B) * 8);
+    f.rest = c.base ? c.base + c.off : nullptr;
+    Carver u(nullptr);
+    carve_update(u, B, N, K, d);
+    c.off += std::max(u.off, ws_assign(B, K, d, dt));
+    return f;
+}
+
+struct HostWs {
+    void *X;
+    float *w, *C;
+    int32_t *ids;
+    double *inertia;
+    void *fit;
+};
+inline HostWs carve_host(Carver &c, int64_t B, int64_t N, int64_t K, int64_t d, km_dtype dt,
+                         bool weighted, int iters) {
+    HostWs h;
+    h.X = c.take<uint8_t>(static_cast<size_t>(B * N * d) * dtype_size(dt));
+    h.w = weighted ? c.take<float>(static_cast<size_t>(B * N) * 4) : nullptr;
+    h.C = c.take<float>(static_cast<size_t>(B * K * d) * 4);
+    h.ids = c.take<int32_t>(static_cast<size_t>(B * N) * 4);
+    h.inertia = c.take<double>(static_cast<size_t>(std::max(iters, 1)) * B * 8);
+    h.fit = c.base ? c.base + c.off : nullptr;
+    carve_fit(c, B, N, K, d, dt);
+    return h;
+}
+
+// ---------------------------------------------------------------- device queries
+
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+    int n = 148;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (dev >= 0 && dev < 64) cache[dev] = n;
+    return n;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+inline km_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? KM_OK : KM_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- kernel launchers
+
+template <typename T>
+km_status run_prep(const float *C, int64_t rows, int64_t d, void *Cx, float *cn, cudaStream_t st) {
+    const int64_t blocks = ceil_div(rows, 8);
+    km::prep_kernel<T><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        C, rows, static_cast<int>(d), static_cast<T *>(Cx), cn);
+    return launch_status();
+}
+
+km_status prep_dispatch(const float *C, km_dtype dt, int64_t rows, int64_t d, void *Cx, float *cn,
+                        cudaStream_t st) {
+    switch (dt) {
+        case KM_F32: return run_prep<float>(C, rows, d, Cx, cn, st);
+        case KM_F16: return run_prep<__half>(C, rows, d, Cx, cn, st);
+        default: return run_prep<__nv_bfloat16>(C, rows, d, Cx, cn, st);
+    }
+}
+
+template <typename T>
+km_status run_finalize(const float *sums, const float *wsum, const int32_t *counts,
+                       const float *C_prev, int64_t rows, int64_t d, float *C_new, void *Cx,
+                       float *cn, cudaStream_t st) {
+    km::finalize_kernel<T><<<static_cast<unsigned>(ceil_div(rows, 8)), 256, 0, st>>>(
+        sums, wsum, counts, C_prev, rows, static_cast<int>(d), C_new, static_cast<T *>(Cx), cn);
+    return launch_status();
+}
+
+km_status finalize_dispatch(const float *sums, const float *wsum, const int32_t *counts,
+                            const float *C_prev, int64_t rows, int64_t d, float *C_new, km_dtype dt,
+                            void *Cx, float *cn, cudaStream_t st) {
+    switch (dt) {
+        case KM_F16: return run_finalize<__half>(sums, wsum, counts, C_prev, rows, d, C_new, Cx, cn, st);
+        case KM_BF16:
+            return run_finalize<__nv_bfloat16>(sums, wsum, counts, C_prev, rows, d, C_new, Cx, cn, st);
+        default: return run_finalize<float>(sums, wsum, counts, C_prev, rows, d, C_new, Cx, cn, st);
+    }
+}
+
+template <typename T>
+km_status run_assign_simt(const void *X, const void *Cx, const float *w, int64_t B, int64_t N,
+                          int64_t K, int64_t d, int32_t *ids, float *mind, double *inertia,
+                          cudaStream_t st) {
+    const T *Xt = static_cast<const T *>(X);
+    const T *Ct = static_cast<const T *>(Cx);
+    for (int64_t b0 = 0; b0 < B; b0 += kMaxGridY) {
+        const int64_t nb = std::min<int64_t>(kMaxGridY, B - b0);
+        dim3 grid(static_cast<unsigned>(ceil_div(N, km::kSimtPts)), static_cast<unsigned>(nb));
+        km::assign_simt_kernel<T><<<grid, km::kSimtPts, 0, st>>>(
+            Xt + b0 * N * d, Ct + b0 * K * d, w ? w + b0 * N : nullptr, static_cast<int>(N),
+            static_cast<int>(K), static_cast<int>(d), ids + b0 * N, mind ? mind + b0 * N : nullptr,
+            inertia ? inertia + b0 : nullptr);
+        if (launch_status() != KM_OK) return KM_ERR_CUDA;
+    }
+    return KM_OK;
+}
+
+template <typename T>
+km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float *cn,
+                        const float *w, int64_t B, int64_t N, int64_t K, int64_t d, int32_t *ids,
+                        float *mind, double *inertia, float *cnp, cudaStream_t st) {
+    using namespace km::tc;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return KM_ERR_CUDA;
+    const int bn = tc_bn(K);
+    const int64_t Kp = tc_kp(K);
+    const int nkc = static_cast<int>(ceil_div(d, KC));
+    km::cnpad_kernel<T><<<static_cast<unsigned>(ceil_div(B * Kp, 8)), 256, 0, st>>>(
+        static_cast<const T *>(Cx), cn, static_cast<int>(B), static_cast<int>(K),
+        static_cast<int>(Kp), static_cast<int>(d), cnp);
+    if (launch_status() != KM_OK) return KM_ERR_CUDA;
+
+    const CUtensorMapDataType tdt =
+        dt == KM_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUtensorMap tmX, tmC;
+    {
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                                    static_cast<cuuint64_t>(B)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(N * d * 2)};
+        const cuuint32_t box[3] = {static_cast<cuuint32_t>(KC), static_cast<cuuint32_t>(BM), 1};
+        if (enc(&tmX, tdt, 3, const_cast<void *>(X), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return KM_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(K),
+                                    static_cast<cuuint64_t>(B)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(K * d * 2)};
+        const cuuint32_t box[3] = {static_cast<cuuint32_t>(KC), static_cast<cuuint32_t>(bn), 1};
+        if (enc(&tmC, tdt, 3, const_cast<void *>(Cx), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return KM_ERR_CUDA;
+    }
+    Params p;
+    p.B = static_cast<int>(B);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.d = static_cast<int>(d);
+    p.nkc = nkc;
+    p.bn = bn;
+    p.nct = static_cast<int>(Kp / bn);
+    p.mtiles = static_cast<int>(ceil_div(N, BM));
+    p.stages = pick_stages(nkc, bn);
+    p.need_xn = (mind || inertia) ? 1 : 0;
+    p.idesc = km::mma_idesc_f16(dt == KM_BF16 ? 1u : 0u, BM, static_cast<uint32_t>(bn));
+    p.cnp = cnp;
+    p.Kp = static_cast<int>(Kp);
+    p.w = w;
+    p.ids = ids;
+    p.mind = mind;
+    p.inertia = inertia;
+    const Layout L = make_layout(nkc, bn, p.stages);
+    // More than half of the shared memory per block keeps one CTA per SM, so no second CTA
+    // ever waits in tcgen05.alloc for the 512 TMEM columns the first one holds.
+    const size_t smem = std::max<size_t>(L.total + 1024, SMEM_LIMIT / 2 + 1024);
+    if (cudaFuncSetAttribute(assign_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return KM_ERR_CUDA;
+    const int64_t items = B * p.mtiles;
+    if (items > kMaxIndex) return KM_ERR_UNSUPPORTED;
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(items, num_sms()));
+    assign_tc_kernel<T><<<grid, NUM_THREADS, smem, st>>>(tmX, tmC, p);
+    return launch_status();
+}
+
+// Validated-argument assignment; `cnp` must hold B * tc_kp(K) floats when the TC path can run.
+km_status do_assign(const void *X, km_dtype dt, const void *Cx, const float *cn, const float *w,
+                    int64_t B, int64_t N, int64_t K, int64_t d, int32_t *ids, float *mind,
+                    double *inertia, float *cnp, cudaStream_t st) {
+    if (inertia && cudaMemsetAsync(inertia, 0, static_cast<size_t>(B) * 8, st) != cudaSuccess)
+        return KM_ERR_CUDA;
+    const bool tc = tc_shape_ok(dt, d) && aligned(X, 16) && aligned(Cx, 16) && cnp != nullptr &&
+                    B * ceil_div(N, 128) <= kMaxIndex;
+    if (tc) {
+        if (dt == KM_F16)
+            return run_assign_tc<__half>(X, dt, Cx, cn, w, B, N, K, d, ids, mind, inertia, cnp, st);
+        return run_assign_tc<__nv_bfloat16>(X, dt, Cx, cn, w, B, N, K, d, ids, mind, inertia, cnp, st);
+    }
+    switch (dt) {
+        case KM_F32: return run_assign_simt<float>(X, Cx, w, B, N, K, d, ids, mind, inertia, st);
+        case KM_F16: return run_assign_simt<__half>(X, Cx, w, B, N, K, d, ids, mind, inertia, st);
+        default: return run_assign_simt<__nv_bfloat16>(X, Cx, w, B, N, K, d, ids, mind, inertia, st);
+    }
+}
+
+template <typename T, int VEC, int G>
+km_status run_segreduce_t(const void *X, const float *w, const int32_t *perm,
+                          const int32_t *offsets, int64_t B, int64_t N, int64_t K, int64_t d,
+                          float *sums, float *wsum, cudaStream_t st) {
+    const int64_t total = B * N;
+    const int64_t target = static_cast<int64_t>(num_sms()) * 48;
+    int64_t range = ceil_div(total, target);
+    range = std::max<int64_t>(256, ceil_div(range, 32) * 32);
+    range = std::min<int64_t>(range, ceil_div(N, 32) * 32);
+    const int64_t rpb = ceil_div(N, range);
+    const int64_t warps = B * rpb;
+    const int64_t ycols = ceil_div(d, static_cast<int64_t>(G) * VEC);
+    dim3 grid(static_cast<unsigned>(ceil_div(warps, km::upd::SEG_THREADS / 32)),
+              static_cast<unsigned>(ycols));
+    if (ycols > kMaxGridY) return KM_ERR_UNSUPPORTED;
+    km::upd::segreduce_kernel<T, VEC, G><<<grid, km::upd::SEG_THREADS, 0, st>>>(
+        static_cast<const T *>(X), w, perm, offsets, static_cast<int>(B), static_cast<int>(N),
+        static_cast<int>(K), static_cast<int>(d), static_cast<int>(range), static_cast<int>(rpb),
+        sums, wsum);
+    return launch_status();
+}
+
+template <typename T, int VEC>
+km_status segreduce_g(int G, const void *X, const float *w, const int32_t *perm,
+                      const int32_t *offsets, int64_t B, int64_t N, int64_t K, int64_t d,
+                      float *sums, float *wsum, cudaStream_t st) {
+    switch (G) {
+        case 1: return run_segreduce_t<T, VEC, 1>(X, w, perm, offsets, B, N, K, d, sums, wsum, st);
+        case 2: return run_segreduce_t<T, VEC, 2>(X, w, perm, offsets, B, N, K, d, sums, wsum, st);
+        case 4: return run_segreduce_t<T, VEC, 4>(X, w, perm, offsets, B, N, K, d, sums, wsum, st);
+        case 8: return run_segreduce_t<T, VEC, 8>(X, w, perm, offsets, B, N, K, d, sums, wsum, st);
+        case 16: return run_segreduce_t<T, VEC, 16>(X, w, perm, offsets, B, N, K, d, sums, wsum, st);
+        default: return run_segreduce_t<T, VEC, 32>(X, w, perm, offsets, B, N, K, d, sums, wsum, st);
+    }
+}
+
+template <typename T>
+km_status segreduce_dispatch(const void *X, const float *w, const int32_t *perm,
+                             const int32_t *offsets, int64_t B, int64_t N, int64_t K, int64_t d,
+                             float *sums, float *wsum, cudaStream_t st) {
+    constexpr int VV = 16 / sizeof(T);
+    const bool vec = (d % VV == 0) && aligned(X, 16) && aligned(sums, 16);
+    const int vw = vec ? VV : 1;
+    int64_t lanes = ceil_div(d, vw);
+    int G = 1;
+    while (G < lanes && G < 32) G <<= 1;
+    if (vec) return segreduce_g<T, VV>(G, X, w, perm, offsets, B, N, K, d, sums, wsum, st);
+    return segreduce_g<T, 1>(G, X, w, perm, offsets, B, N, K, d, sums, wsum, st);
+}
+
+// sums[B,K,d], counts[B,K] and (when non-null) wsum[B,K] are overwritten.
+km_status do_update_partial(const void *X, km_dtype dt, const int32_t *ids, const float *w,
+                            int64_t B, int64_t N, int64_t K, int64_t d, float *sums, float *wsum,
+                            int32_t *counts, const UpdateWs &u, cudaStream_t st) {
+    if (cudaMemsetAsync(counts, 0, static_cast<size_t>(B * K) * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(sums, 0, static_cast<size_t>(B * K * d) * 4, st) != cudaSuccess ||
+        (wsum && cudaMemsetAsync(wsum, 0, static_cast<size_t>(B * K) * 4, st) != cudaSuccess))
+        return KM_ERR_CUDA;
+    using namespace km::upd;
+    const bool smem_bins = K <= SMEM_K_MAX;
+    const int64_t ntiles = ceil_div(N, TILE);
+    for (int64_t b0 = 0; b0 < B; b0 += kMaxGridY) {
+        const int64_t nb = std::min<int64_t>(kMaxGridY, B - b0);
+        dim3 grid(static_cast<unsigned>(ntiles), static_cast<unsigned>(nb));
+        hist_kernel<<<grid, TILE_THREADS, smem_bins ? K * 4 : 0, st>>>(
+            ids + b0 * N, static_cast<int>(N), static_cast<int>(K), counts + b0 * K, smem_bins);
+        if (launch_status() != KM_OK) return KM_ERR_CUDA;
+    }
+    scan_kernel<<<static_cast<unsigned>(B), SCAN_THREADS, 0, st>>>(counts, static_cast<int>(K),
+                                                                      u.offsets, u.cursor);
+    if (launch_status() != KM_OK) return KM_ERR_CUDA;
+    const size_t scatter_smem = smem_bins ? static_cast<size_t>(K + TILE) * 4 : 0;
+    if (smem_bins && cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(scatter_smem)) != cudaSuccess)
+        return KM_ERR_CUDA;
+    if (smem_bins && cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(K * 4)) != cudaSuccess)
+        return KM_ERR_CUDA;
+    for (int64_t b0 = 0; b0 < B; b0 += kMaxGridY) {
+        const int64_t nb = std::min<int64_t>(kMaxGridY, B - b0);
+        dim3 grid(static_cast<unsigned>(ntiles), static_cast<unsigned>(nb));
+        scatter_kernel<<<grid, TILE_THREADS, scatter_smem, st>>>(
+            ids + b0 * N, static_cast<int>(N), static_cast<int>(K), u.cursor + b0 * K,
+            u.perm + b0 * N, smem_bins);
+        if (launch_status() != KM_OK) return KM_ERR_CUDA;
+    }
+    switch (dt) {
+        case KM_F32: return segreduce_dispatch<float>(X, w, u.perm, u.offsets, B, N, K, d, sums, wsum, st);
+        case KM_F16: return segreduce_dispatch<__half>(X, w, u.perm, u.offsets, B, N, K, d, sums, wsum, st);
+        default:
+            return segreduce_dispatch<__nv_bfloat16>(X, w, u.perm, u.offsets, B, N, K, d, sums, wsum, st);
+    }
+}
+
+template <typename T>
+km_status run_fit1d(const void *X, const float *w, int64_t B, int64_t N, int64_t K, float *C,
+                    int iters, int32_t *ids, double *inertia_hist, float *C_hist, cudaStream_t st) {
+    int NP = 2;
+    while (NP < N) NP <<= 1;
+    const size_t smem = static_cast<size_t>(NP) * 12;
+    if (cudaFuncSetAttribute(km::fit1d::fit1d_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return KM_ERR_CUDA;
+    km::fit1d::fit1d_kernel<T><<<static_cast<unsigned>(B), km::fit1d::THREADS, smem, st>>>(
+        static_cast<const T *>(X), w, static_cast<int>(B), static_cast<int>(N), NP,
+        static_cast<int>(K), iters, C, ids, inertia_hist, C_hist);
+    return launch_status();
+}
+
+inline bool fit1d_ok(int64_t N, int64_t K, int64_t d) {
+    return d == 1 && K <= km::fit1d::KMAX && N <= km::fit1d::NMAX;
+}
+
+km_status do_fit(const void *X, km_dtype dt, const float *w, int64_t B, int64_t N, int64_t K,
+                 int64_t d, float *C, int iters, int32_t *ids, double *inertia_hist, float *C_hist,
+                 void *ws, cudaStream_t st) {
+    if (fit1d_ok(N, K, d)) {
+        switch (dt) {
+            case KM_F32: return run_fit1d<float>(X, w, B, N, K, C, iters, ids, inertia_hist, C_hist, st);
+            case KM_F16: return run_fit1d<__half>(X, w, B, N, K, C, iters, ids, inertia_hist, C_hist, st);
+            default:
+                return run_fit1d<__nv_bfloat16>(X, w, B, N, K, C, iters, ids, inertia_hist, C_hist, st);
+        }
+    }
+    Carver c(ws);
+    FitWs f = carve_fit(c, B, N, K, d, dt);
+    Carver r(f.rest);
+    UpdateWs u = carve_update(r, B, N, K, d);
+    float *cnp = static_cast<float *>(f.rest);  // assignment scratch shares the update region
+    const size_t cbytes = static_cast<size_t>(B * K * d) * 4;
+    km_status s = prep_dispatch(C, dt, B * K, d, f.Cx, f.cn, st);
+    if (s != KM_OK) return s;
+    for (int t = 0; t < iters; ++t) {
+        if (C_hist && cudaMemcpyAsync(C_hist + static_cast<int64_t>(t) * B * K * d, C, cbytes,
+                                      cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+            return KM_ERR_CUDA;
+        double *in = inertia_hist ? inertia_hist + static_cast<int64_t>(t) * B : nullptr;
+        s = do_assign(X, dt, f.Cx, f.cn, w, B, N, K, d, f.ids, nullptr, in, cnp, st);
+        if (s != KM_OK) return s;
+        s = do_update_partial(X, dt, f.ids, w, B, N, K, d, u.sums, w ? u.wsum : nullptr, f.counts, u, st);
+        if (s != KM_OK) return s;
+        s = finalize_dispatch(u.sums, w ? u.wsum : nullptr, f.counts, C, B * K, d, C, dt, f.Cx, f.cn, st);
+        if (s != KM_OK) return s;
+    }
+    if (C_hist && cudaMemcpyAsync(C_hist + static_cast<int64_t>(iters) * B * K * d, C, cbytes,
+                                  cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return KM_ERR_CUDA;
+    if (ids) return do_assign(X, dt, f.Cx, f.cn, w, B, N, K, d, ids, nullptr, nullptr, cnp, st);
+    return KM_OK;
+}
+
+inline bool elem_aligned(const void *p, km_dtype dt) { return aligned(p, dtype_size(dt)); }
+
+}  // namespace
+
+// =================================================================== exported C ABI
+
+extern "C" {
+
+const char *km_status_string(km_status s) {
+    switch (s) {
+        case KM_OK: return "KM_OK";
+        case KM_ERR_INVALID_ARG: return "KM_ERR_INVALID_ARG";
+        case KM_ERR_UNSUPPORTED: return "KM_ERR_UNSUPPORTED";
+        case KM_ERR_WORKSPACE: return "KM_ERR_WORKSPACE";
+        case KM_ERR_CUDA: return "KM_ERR_CUDA";
+        case KM_ERR_DEVICE_TIMEOUT: return "KM_ERR_DEVICE_TIMEOUT";
+    }
+    return "KM_ERR_UNKNOWN";
+}
+
+int km_abi_version(void) { return 1; }
+
+int km_assign_uses_tensor_cores(km_dtype dtype, int64_t d, const void *X, const void *Cx) {
+    return valid_dtype(dtype) && tc_shape_ok(dtype, d) && aligned(X, 16) && aligned(Cx, 16) ? 1 : 0;
+}
+
+size_t km_workspace_size(km_op op, int64_t B, int64_t N, int64_t K, int64_t d, km_dtype dtype,
+                         int weighted, int iters) {
+    if (!sizes_ok(B, N, K, d) || !valid_dtype(dtype) || iters < 0) return 0;
+    Carver c(nullptr);
+    switch (op) {
+        case KM_OP_ASSIGN: return ws_assign(B, K, d, dtype);
+        case KM_OP_UPDATE: carve_update(c, B, N, K, d); return c.off;
+        case KM_OP_FIT: carve_fit(c, B, N, K, d, dtype); return c.off;
+        case KM_OP_FIT_HOST: carve_host(c, B, N, K, d, dtype, weighted != 0, iters); return c.off;
+    }
+    return 0;
+}
+
+km_status km_prep(const float *C, km_dtype dtype, int64_t B, int64_t K, int64_t d, void *Cx,
+                  float *cn, void *stream) {
+    if (!C || (!Cx && !cn) || !valid_dtype(dtype) || !sizes_ok(B, 1, K, d) || !aligned(C, 4) ||
+        (Cx && !elem_aligned(Cx, dtype)) || (cn && !aligned(cn, 4)))
+        return KM_ERR_INVALID_ARG;
+    return prep_dispatch(C, dtype, B * K, d, Cx, cn, S(stream));
+}
+
+km_status km_assign(const void *X, km_dtype dtype, const void *Cx, const float *cn, const float *w,
+                    int64_t B, int64_t N, int64_t K, int64_t d, int32_t *ids, float *mind,
+                    double *inertia, void *ws, size_t ws_bytes, void *stream) {
+    if (!X || !Cx || !ids || !valid_dtype(dtype) || !sizes_ok(B, N, K, d) ||
+        !elem_aligned(X, dtype) || !elem_aligned(Cx, dtype) || !aligned(ids, 4) ||
+        (w && !aligned(w, 4)) || (cn && !aligned(cn, 4)) || (mind && !aligned(mind, 4)) ||
+        (inertia && !aligned(inertia, 8)))
+        return KM_ERR_INVALID_ARG;
+    const size_t need = ws_assign(B, K, d, dtype);
+    if (need && (!ws || ws_bytes < need || !aligned(ws, kAlign))) return KM_ERR_WORKSPACE;
+    return do_assign(X, dtype, Cx, cn, w, B, N, K, d, ids, mind, inertia,
+                     need ? static_cast<float *>(ws) : nullptr, S(stream));
+}
+
+km_status km_update_partial(const void *X, km_dtype dtype, const int32_t *ids, const float *w,
+                            int64_t B, int64_t N, int64_t K, int64_t d, float *sums, float *wsum,
+                            int32_t *counts, void *ws, size_t ws_bytes, void *stream) {
+    if (!X || !ids || !sums || !counts || !valid_dtype(dtype) || !sizes_ok(B, N, K, d) ||
+        !elem_aligned(X, dtype) || !aligned(ids, 4) || !aligned(sums, 4) || !aligned(counts, 4) ||
+        (w && !aligned(w, 4)) || (wsum && !aligned(wsum, 4)) || (w && !wsum))
+        return KM_ERR_INVALID_ARG;
+    Carver c(nullptr);
+    carve_update(c, B, N, K, d);
+    if (!ws || ws_bytes < c.off || !aligned(ws, kAlign)) return KM_ERR_WORKSPACE;
+    Carver r(ws);
+    UpdateWs u = carve_update(r, B, N, K, d);
+    return do_update_partial(X, dtype, ids, w, B, N, K, d, sums, wsum, counts, u, S(stream));
+}
+
+km_status km_finalize(const float *sums, const float *wsum, const int32_t *counts,
+                      const float *C_prev, int64_t B, int64_t K, int64_t d, float *C_new,
+                      km_dtype cx_dtype, void *Cx, float *cn, void *stream) {
+    if (!sums || !counts || !C_prev || !C_new || !sizes_ok(B, 1, K, d) || !valid_dtype(cx_dtype) ||
+        (Cx && !elem_aligned(Cx, cx_dtype)))
+        return KM_ERR_INVALID_ARG;
+    return finalize_dispatch(sums, wsum, counts, C_prev, B * K, d, C_new, Cx ? cx_dtype : KM_F32,
+                             Cx, cn, S(stream));
+}
+
+km_status km_update(const void *X, km_dtype dtype, const int32_t *ids, const float *w, int64_t B,
+                    int64_t N, int64_t K, int64_t d, const float *C_prev, float *C_new,
+                    int32_t *counts, float *wsum, void *ws, size_t ws_bytes, void *stream) {
+    if (!X || !ids || !C_prev || !C_new || !counts || !valid_dtype(dtype) || !sizes_ok(B, N, K, d) ||
+        !elem_aligned(X, dtype) || !aligned(ids, 4) || !aligned(counts, 4) || !aligned(C_prev, 4) ||
+        !aligned(C_new, 4) || (w && !aligned(w, 4)) || (wsum && !aligned(wsum, 4)))
+        return KM_ERR_INVALID_ARG;
+    Carver c(nullptr);
+    carve_update(c, B, N, K, d);
+    if (!ws || ws_bytes < c.off || !aligned(ws, kAlign)) return KM_ERR_WORKSPACE;
+    Carver r(ws);
+    UpdateWs u = carve_update(r, B, N, K, d);
+    float *ws_w = wsum ? wsum : (w ? u.wsum : nullptr);
+    km_status s = do_update_partial(X, dtype, ids, w, B, N, K, d, u.sums, ws_w, counts, u, S(stream));
+    if (s != KM_OK) return s;
+    return finalize_dispatch(u.sums, w ? ws_w : nullptr, counts, C_prev, B * K, d, C_new, KM_F32,
+                             nullptr, nullptr, S(stream));
+}
+
+km_status km_init_grid1d(const void *X, km_dtype dtype, int64_t B, int64_t N, int64_t K, float *C,
+                         void *stream) {
+    if (!X || !C || !valid_dtype(dtype) || !sizes_ok(B, N, K, 1) || !elem_aligned(X, dtype) ||
+        !aligned(C, 4))
+        return KM_ERR_INVALID_ARG;
+    const unsigned grid = static_cast<unsigned>(B);
+    switch (dtype) {
+        case KM_F32:
+            km::fit1d::grid_init_kernel<float><<<grid, 256, 0, S(stream)>>>(
+                static_cast<const float *>(X), static_cast<int>(N), static_cast<int>(K), C);
+            break;
+        case KM_F16:
+            km::fit1d::grid_init_kernel<__half><<<grid, 256, 0, S(stream)>>>(
+                static_cast<const __half *>(X), static_cast<int>(N), static_cast<int>(K), C);
+            break;
+        default:
+            km::fit1d::grid_init_kernel<__nv_bfloat16><<<grid, 256, 0, S(stream)>>>(
+                static_cast<const __nv_bfloat16 *>(X), static_cast<int>(N), static_cast<int>(K), C);
+    }
+    return launch_status();
+}
+
+km_status km_fit(const void *X, km_dtype dtype, const float *w, int64_t B, int64_t N, int64_t K,
+                 int64_t d, float *C, int iters, int32_t *ids, double *inertia_hist, float *C_hist,
+                 void *ws, size_t ws_bytes, void *stream) {
+    if (!X || !C || iters < 0 || !valid_dtype(dtype) || !sizes_ok(B, N, K, d) ||
+        !elem_aligned(X, dtype) || !aligned(C, 4) || (w && !aligned(w, 4)) ||
+        (ids && !aligned(ids, 4)) || (inertia_hist && !aligned(inertia_hist, 8)) ||
+        (C_hist && !aligned(C_hist, 4)))
+        return KM_ERR_INVALID_ARG;
+    if (!fit1d_ok(N, K, d)) {
+        Carver c(nullptr);
+        carve_fit(c, B, N, K, d, dtype);
+        if (!ws || ws_bytes < c.off || !aligned(ws, kAlign)) return KM_ERR_WORKSPACE;
+    }
+    return do_fit(X, dtype, w, B, N, K, d, C, iters, ids, inertia_hist, C_hist, ws, S(stream));
+}
+
+km_status km_fit_host(const void *X_host, km_dtype dtype, const float *w_host, int64_t B,
+                      int64_t N, int64_t K, int64_t d, float *C_host, int iters, int32_t *ids_host,
+                      double *inertia_host, void *ws, size_t ws_bytes, void *stream) {
+    if (!X_host || !C_host || iters < 0 || !valid_dtype(dtype) || !sizes_ok(B, N, K, d))
+        return KM_ERR_INVALID_ARG;
+    Carver c(nullptr);
+    carve_host(c, B, N, K, d, dtype, w_host != nullptr, iters);
+    if (!ws || ws_bytes < c.off || !aligned(ws, kAlign)) return KM_ERR_WORKSPACE;
+    Carver r(ws);
+    HostWs h = carve_host(r, B, N, K, d, dtype, w_host != nullptr, iters);
+    cudaStream_t st = S(stream);
+    const size_t xb = static_cast<size_t>(B * N * d) * dtype_size(dtype);
+    const size_t cb = static_cast<size_t>(B * K * d) * 4;
+    if (cudaMemcpyAsync(h.X, X_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        (w_host && cudaMemcpyAsync(h.w, w_host, static_cast<size_t>(B * N) * 4,
+                                   cudaMemcpyHostToDevice, st) != cudaSuccess) ||
+        cudaMemcpyAsync(h.C, C_host, cb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return KM_ERR_CUDA;
+    km_status s = do_fit(h.X, dtype, w_host ? h.w : nullptr, B, N, K, d, h.C, iters,
+                         ids_host ? h.ids : nullptr, (inertia_host && iters) ? h.inertia : nullptr,
+                         nullptr, h.fit, st);
+    if (s != KM_OK) return s;
+    if (cudaMemcpyAsync(C_host, h.C, cb, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        (ids_host && cudaMemcpyAsync(ids_host, h.ids, static_cast<size_t>(B * N) * 4,
+                                     cudaMemcpyDeviceToHost, st) != cudaSuccess) ||
+        (inertia_host && iters &&
+         cudaMemcpyAsync(inertia_host, h.inertia, static_cast<size_t>(iters) * B * 8,
+                         cudaMemcpyDeviceToHost, st) != cudaSuccess))
+        return KM_ERR_CUDA;
+    return cudaStreamSynchronize(st) == cudaSuccess ? KM_OK : KM_ERR_CUDA;
+}
+
+km_status km_device_error(void *stream, int *code) {
+    if (!code) return KM_ERR_INVALID_ARG;
+    *code = 0;
+    if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return KM_ERR_CUDA;
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, km::g_km_dev_error, sizeof(v)) != cudaSuccess ||
+        cudaMemcpyToSymbol(km::g_km_dev_error, &zero, sizeof(zero)) != cudaSuccess)
+        return KM_ERR_CUDA;
+    *code = static_cast<int>(v);
+    return v ? KM_ERR_DEVICE_TIMEOUT : KM_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,191 @@
+/*
+ * kmeans_b200.h -- C ABI of libkmeans_b200.so: exact Lloyd k-means on NVIDIA B200 (sm_100a).
+ *
+ * One Lloyd iteration has two stages (technologypulse.uk "Flash-KMeans" article, section
+ * "Flash-KMeans: same maths, new dataflow"; wispaper.ai Flash-KMeans blog, Background):
+ *   assignment  ids[i] = argmin_k ||x_i - c_k||^2
+ *   update      c_k    = (sum_{i: ids[i]=k} w_i x_i) / (sum_{i: ids[i]=k} w_i)
+ * The assignment never materialises the N x K distance matrix (FlashAssign, same article,
+ * "Bottleneck 1"; wispaper blog "1. FlashAssign"). The update sorts the assignment vector so
+ * that each cluster's points form one contiguous segment and reduces segment by segment, with
+ * one atomic merge per segment instead of one per point (Sort-Inverse Update, same article,
+ * "Bottleneck 2"; wispaper blog "2. Sort-Inverse Update"). Per-point sample weights and the
+ * uniform-grid initialisation linspace(min, max, K) come from the per-row 1-D codebook fitting
+ * of the LeanQuant issue "1D k-means" (kmeans_fit with sample_weight).
+ *
+ * Conventions for every entry point:
+ *   - Layout: row-major, innermost index last. X[B,N,d], C[B,K,d], w[B,N], ids[B,N],
+ *     cn[B,K], counts[B,K]. B independent problems ("batches") share nothing.
+ *   - Pointers are DEVICE pointers owned by the caller, except in km_fit_host (host pointers,
+ *     see there). The library allocates no memory: scratch comes from the caller's workspace,
+ *     sized by km_workspace_size. Nothing is retained between calls.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call only enqueues work
+ *     on that stream and returns; KM_OK means "validated and enqueued". km_fit_host is the one
+ *     synchronous call.
+ *   - Argument errors are reported synchronously, before anything is enqueued:
+ *     KM_ERR_INVALID_ARG (null required pointer, a size <= 0, N or K >= 2^31, misaligned
+ *     pointer), KM_ERR_UNSUPPORTED (dtype/shape combination not provided), KM_ERR_WORKSPACE
+ *     (workspace smaller than km_workspace_size). A failed launch returns KM_ERR_CUDA.
+ *   - Device-side waits in the kernels are bounded; a wait that runs out records an error word
+ *     on the device and the kernel exits. km_device_error() reads and clears it.
+ *   - Numerics: fp16/bf16/fp32 inputs, fp32 accumulation, fp32 master centroids. The
+ *     assignment compares distances to the centroids rounded (round-to-nearest-even) to X's
+ *     dtype, with ||c||^2 computed from the rounded values; ties go to the lowest index.
+ *     Inputs containing NaN or Inf give undefined results.
+ *   - Empty clusters (count 0 or total weight 0) keep their previous centroid.
+ */
+#ifndef KMEANS_B200_H
+#define KMEANS_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum km_status {
+    KM_OK = 0,
+    KM_ERR_INVALID_ARG = 1,
+    KM_ERR_UNSUPPORTED = 2,
+    KM_ERR_WORKSPACE = 3,
+    KM_ERR_CUDA = 4,
+    KM_ERR_DEVICE_TIMEOUT = 5
+} km_status;
+
+typedef enum km_dtype { KM_F32 = 0, KM_F16 = 1, KM_BF16 = 2 } km_dtype;
+
+typedef enum km_op { KM_OP_ASSIGN = 0, KM_OP_UPDATE = 1, KM_OP_FIT = 2, KM_OP_FIT_HOST = 3 } km_op;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *km_status_string(km_status s);
+
+/* ABI version of this library (incremented on any signature change). */
+int km_abi_version(void);
+
+/*
+ * Bytes of device workspace the entry point `op` needs for these sizes (0 on invalid sizes, and
+ * 0 for KM_OP_ASSIGN when the CUDA-core path needs none). `weighted` != 0 when a weight array
+ * will be passed and `iters` the iteration count (both matter for KM_OP_FIT_HOST only).
+ * The workspace must be 256-byte aligned; its contents need not be initialised.
+ */
+size_t km_workspace_size(km_op op, int64_t B, int64_t N, int64_t K, int64_t d, km_dtype dtype,
+                         int weighted, int iters);
+
+/*
+ * Centroid preparation for the assignment: Cx[b,k,:] = C[b,k,:] rounded to `dtype` (RNE), and
+ * cn[b,k] = sum_j Cx[b,k,j]^2 in fp32 from the rounded values (the ||c||^2 term of the expanded
+ * distance ||x||^2 - 2<x,c> + ||c||^2 used by FlashAssign; technologypulse.uk Flash-KMeans
+ * article, "Bottleneck 1"). C[B,K,d] fp32 in; Cx[B,K,d] in `dtype`, cn[B,K] fp32 out.
+ */
+km_status km_prep(const float *C, km_dtype dtype, int64_t B, int64_t K, int64_t d, void *Cx,
+                  float *cn, void *stream);
+
+/*
+ * Assignment stage (FlashAssign): ids[b,i] = argmin_k ||X[b,i,:] - Cx[b,k,:]||^2, lowest k on
+ * ties, computed tile by tile with a running (min, argmin) per point so that no N x K matrix is
+ * written (technologypulse.uk Flash-KMeans article, "Bottleneck 1"; wispaper blog
+ * "1. FlashAssign", online argmin).
+ *   X[B,N,d] in `dtype`; Cx[B,K,d] in the same dtype (see km_prep);
+ *   cn[B,K] fp32 = ||Cx[b,k]||^2, or NULL (then computed into the workspace);
+ *   w[B,N] fp32 per-point weights for the inertia, or NULL (all ones);
+ *   ids[B,N] int32 out (required); mind[B,N] fp32 out or NULL: the squared distance to the
+ *   chosen centroid, max(0, .); inertia[B] fp64 out or NULL: sum_i w_i * mind_i.
+ * fp16/bf16 with d % 8 == 0, 8 <= d <= 256 and 16-byte aligned X/Cx run on the tcgen05 tensor
+ * cores (fp32 accumulation of <x,c>); every other case runs an exact-fp32 CUDA-core kernel that
+ * evaluates sum_j (x_j - c_j)^2 directly.
+ */
+km_status km_assign(const void *X, km_dtype dtype, const void *Cx, const float *cn,
+                    const float *w, int64_t B, int64_t N, int64_t K, int64_t d, int32_t *ids,
+                    float *mind, double *inertia, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * 1 when km_assign with these arguments runs on the tcgen05 tensor cores, 0 when it runs the
+ * exact-fp32 CUDA-core kernel (no launch, no validation beyond the eligibility rule).
+ */
+int km_assign_uses_tensor_cores(km_dtype dtype, int64_t d, const void *X, const void *Cx);
+
+/*
+ * Update stage (Sort-Inverse Update), fed an assignment ids[B,N] (values in [0,K)):
+ *   counts[b,k] = #{i : ids[b,i] = k}                                        (int32, required)
+ *   wsum[b,k]   = sum of w over those points (fp32; NULL allowed)
+ *   C_new[b,k]  = sum_i w_i X[b,i,:] / wsum[b,k], or C_prev[b,k] when the cluster is empty.
+ * The ids are argsorted per batch by a device counting sort into contiguous per-cluster
+ * segments; X is read in sorted order by index (never permuted in memory) and each chunk of
+ * sorted positions reduces its runs on chip, merging each run with one vector atomic per
+ * coordinate block (technologypulse.uk Flash-KMeans article, "Bottleneck 2"; wispaper blog
+ * "2. Sort-Inverse Update"). C_new may alias C_prev. Points whose id lies outside [0,K) are
+ * ignored (neither counted nor summed).
+ */
+km_status km_update(const void *X, km_dtype dtype, const int32_t *ids, const float *w, int64_t B,
+                    int64_t N, int64_t K, int64_t d, const float *C_prev, float *C_new,
+                    int32_t *counts, float *wsum, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * First half of km_update, for callers that combine partial sums across devices (points
+ * split over GPUs, centroids replicated): writes this device's sums[B,K,d] (fp32,
+ * sum_i w_i x_i), wsum[B,K] (fp32, may be NULL when w is NULL) and counts[B,K] (int32), all
+ * overwritten (not accumulated). Same sort-inverse reduction as km_update. Uses the
+ * KM_OP_UPDATE workspace.
+ */
+km_status km_update_partial(const void *X, km_dtype dtype, const int32_t *ids, const float *w,
+                            int64_t B, int64_t N, int64_t K, int64_t d, float *sums, float *wsum,
+                            int32_t *counts, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Second half of km_update: C_new[b,k] = sums[b,k] / wsum[b,k] (wsum NULL: counts) when
+ * counts[b,k] > 0 and the divisor is > 0, else C_prev[b,k] (the mean S_j / N_j of the e-means
+ * daily's Lloyd recap, steinslab, first section). Optionally also writes Cx (C_new rounded to
+ * `cx_dtype`) and cn = ||Cx||^2 for the next assignment (pass NULL to skip). C_new may alias
+ * C_prev.
+ */
+km_status km_finalize(const float *sums, const float *wsum, const int32_t *counts,
+                      const float *C_prev, int64_t B, int64_t K, int64_t d, float *C_new,
+                      km_dtype cx_dtype, void *Cx, float *cn, void *stream);
+
+/*
+ * Uniform-grid initialisation of 1-D rows (LeanQuant issue "1D k-means": the sklearn init
+ * np.linspace(row.min(), row.max(), K)): with lo/hi the min/max of X[b,:,0],
+ * C[b,k] = k * ((hi - lo) / (K - 1)) + lo evaluated in fp64 exactly as numpy's linspace does,
+ * C[b,K-1] = hi, K == 1 gives lo; then rounded to fp32. X[B,N,1] in `dtype`, C[B,K] fp32 out.
+ */
+km_status km_init_grid1d(const void *X, km_dtype dtype, int64_t B, int64_t N, int64_t K, float *C,
+                         void *stream);
+
+/*
+ * `iters` Lloyd iterations from the centroids in C[B,K,d] (fp32, in/out), then (only when ids is
+ * non-NULL) one final assignment against the final centroids written to ids[B,N].
+ *   inertia_hist[iters,B] fp64 out or NULL: inertia of iteration t's assignment;
+ *   C_hist[iters+1,B,K,d] fp32 out or NULL: the centroids entering each iteration and the final
+ *   ones (C_hist[0] = the input C).
+ * d == 1 with K <= 64 and N <= 8192 runs one fused kernel per row that keeps the row and its
+ * weights on chip for all iterations (the per-row codebook setting of the LeanQuant issue);
+ * everything else chains km_prep / km_assign / km_update on the stream.
+ */
+km_status km_fit(const void *X, km_dtype dtype, const float *w, int64_t B, int64_t N, int64_t K,
+                 int64_t d, float *C, int iters, int32_t *ids, double *inertia_hist,
+                 float *C_hist, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * km_fit on HOST buffers: copies X_host (and w_host, C_host) to the device staging area inside
+ * the workspace (one cudaMemcpyAsync per array), runs km_fit, copies C back into C_host and,
+ * when non-NULL, ids into ids_host[B,N] and the inertia history into inertia_host[iters,B],
+ * then synchronises `stream`. Host buffers should be pinned for full PCIe bandwidth. The
+ * workspace (device memory) is sized by km_workspace_size(KM_OP_FIT_HOST, ..., weighted, iters).
+ */
+km_status km_fit_host(const void *X_host, km_dtype dtype, const float *w_host, int64_t B,
+                      int64_t N, int64_t K, int64_t d, float *C_host, int iters, int32_t *ids_host,
+                      double *inertia_host, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word of the current device.
+ * *code = 0 when no kernel recorded an error; otherwise a bit mask (1 = a bounded wait ran out).
+ * Returns KM_ERR_DEVICE_TIMEOUT when *code != 0, KM_ERR_CUDA when the synchronisation failed.
+ */
+km_status km_device_error(void *stream, int *code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KMEANS_B200_H */

@@ -1,0 +1,267 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI (needs a B200).
+
+Sizes are chosen so the oracle finishes in seconds while the kernels still see several tiles
+and ragged tails (N not a multiple of 128, K not a multiple of the centroid tile, d not a
+multiple of 64). Full-size workloads are in test_gpu_fullsize.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import exact_lloyd_means_assign_b200 as km
+import oracle
+import synth
+from parity import check_assign, check_update, mixture, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device(cuda_device):
+    torch.cuda.set_device(cuda_device)
+    yield
+    assert km.km_device_error() == 0
+
+
+DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+
+
+# ------------------------------------------------------------------ prep / grid init
+
+@pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
+def test_prep_rounds_and_norms(dt, cuda_device):
+    dtype = DT[dt]
+    C = torch.randn((3, 50, 40), device=cuda_device) * 3
+    Cx, cn = km.km_prep(C, dtype)
+    torch.cuda.synchronize()
+    assert torch.equal(Cx, C.to(dtype))
+    ref = (Cx.double() ** 2).sum(-1)
+    torch.testing.assert_close(cn.double(), ref, rtol=2e-6, atol=0)
+
+
+@pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("K", [1, 2, 8, 16, 33])
+def test_grid_init_matches_oracle(dt, K, cuda_device):
+    g = torch.Generator().manual_seed(K)
+    X = (torch.randn((37, 1001, 1), generator=g) * 0.02).to(DT[dt])
+    C = km.km_init_grid1d(X.to(cuda_device), K)
+    ref = oracle.grid_init(X, K).astype(np.float32)
+    np.testing.assert_array_equal(to_np(C), ref)
+
+
+# ------------------------------------------------------------------ assignment
+
+TC_CASES = [
+    ("f16", 2, 3000, 300, 128),
+    ("bf16", 2, 3000, 300, 128),
+    ("f16", 1, 1000, 1024, 128),
+    ("f16", 3, 777, 64, 64),
+    ("f16", 2, 500, 100, 96),
+    ("f16", 1, 640, 200, 16),
+    ("f16", 1, 300, 37, 200),
+    ("bf16", 1, 300, 513, 256),
+    ("f16", 1, 129, 1, 128),
+    ("f16", 2, 100, 300, 24),
+    ("bf16", 5, 1, 7, 8),
+]
+SIMT_CASES = [
+    ("f32", 1, 4096, 32, 16),
+    ("f16", 2, 1000, 50, 12),
+    ("f32", 1, 500, 70, 130),
+    ("bf16", 1, 300, 40, 1),
+    ("f16", 1, 200, 20, 264),
+]
+
+
+@pytest.mark.parametrize("dt,B,N,K,d", TC_CASES + SIMT_CASES)
+@pytest.mark.parametrize("weighted", [False, True])
+def test_assign_matches_oracle(dt, B, N, K, d, weighted, cuda_device):
+    dtype = DT[dt]
+    X, C = mixture(B, N, d, K, dtype, cuda_device, seed=B * 1000 + N + K + d)
+    w = (torch.rand((B, N), device=cuda_device) + 0.1) if weighted else None
+    Cx, cn = km.km_prep(C, dtype)
+    assert km.km_assign_uses_tensor_cores(X, Cx) == ((dt, B, N, K, d) in TC_CASES)
+    ids, mind, inertia = km.km_assign(X, Cx, cn, w=w, want_mind=True, want_inertia=True)
+    torch.cuda.synchronize()
+    near = check_assign(X, C, ids, w=w, mind_gpu=mind, inertia_gpu=inertia)
+    assert near <= max(2, B * N // 200)
+    # without cn the kernel computes the norms itself; without mind/inertia it skips ||x||^2
+    ids2, _, _ = km.km_assign(X, Cx)
+    torch.cuda.synchronize()
+    check_assign(X, C, ids2)
+
+
+@pytest.mark.parametrize("dt,d", [("f16", 128), ("bf16", 64), ("f32", 16), ("f16", 12)])
+def test_duplicate_centroids_go_to_lowest_index(dt, d, cuda_device):
+    dtype = DT[dt]
+    X, C = mixture(1, 2000, d, 300, dtype, cuda_device, seed=5)
+    C[0, 290] = C[0, 3]      # duplicates in different centroid tiles
+    C[0, 150] = C[0, 3]
+    Cx, cn = km.km_prep(C, dtype)
+    ids, _, _ = km.km_assign(X, Cx, cn)
+    torch.cuda.synchronize()
+    g = to_np(ids)
+    assert not (g == 290).any() and not (g == 150).any()
+    ids_ref, d1, d2, _ = oracle.assign(oracle.as_f64(X.cpu()), oracle.round_to_dtype(C.cpu(), dtype))
+    np.testing.assert_array_equal(g[ids_ref == 3], 3)
+
+
+def test_all_points_identical(cuda_device):
+    X = torch.full((1, 700, 128), 0.5, dtype=torch.float16, device=cuda_device)
+    C = torch.randn((1, 300, 128), device=cuda_device)
+    C[0, 123] = 0.5
+    Cx, cn = km.km_prep(C, torch.float16)
+    ids, mind, _ = km.km_assign(X, Cx, cn, want_mind=True)
+    torch.cuda.synchronize()
+    assert (ids == 123).all()
+    assert float(mind.max()) < 1e-2
+
+
+# ------------------------------------------------------------------ update
+
+UPD_CASES = [
+    ("f16", 2, 3000, 300, 128),
+    ("bf16", 1, 5000, 64, 64),
+    ("f32", 1, 4096, 32, 16),
+    ("f16", 3, 1000, 50, 12),
+    ("f16", 1, 800, 20, 300),
+    ("f32", 2, 600, 17, 1),
+    ("f16", 1, 100, 400, 128),       # K > N: empty clusters keep their centroid
+    ("f16", 1, 20000, 3, 32),        # few huge segments spanning many warps
+]
+
+
+@pytest.mark.parametrize("dt,B,N,K,d", UPD_CASES)
+@pytest.mark.parametrize("weighted", [False, True])
+def test_update_matches_oracle(dt, B, N, K, d, weighted, cuda_device):
+    dtype = DT[dt]
+    X, C = mixture(B, N, d, K, dtype, cuda_device, seed=N + K)
+    w = (torch.rand((B, N), device=cuda_device) * 2 + 0.01) if weighted else None
+    Cx, cn = km.km_prep(C, dtype)
+    ids, _, _ = km.km_assign(X, Cx, cn)
+    C_new, counts, wsum = km.km_update(X, ids, C, w=w, want_wsum=True)
+    torch.cuda.synchronize()
+    check_update(X, ids, C, C_new, counts, w=w, wsum_gpu=wsum)
+    # partial + finalize is the same computation split in two
+    sums, ws2, c2 = km.km_update_partial(X, ids, K, w=w)
+    C2, Cx2, cn2 = km.km_finalize(sums, c2, C, wsum=ws2, cx_dtype=dtype)
+    torch.cuda.synchronize()
+    assert torch.equal(c2, counts)
+    torch.testing.assert_close(C2, C_new, rtol=1e-5, atol=1e-6)
+    assert torch.equal(Cx2, C2.to(dtype))
+
+
+def test_update_in_place_and_random_ids(cuda_device):
+    g = torch.Generator().manual_seed(3)
+    X = torch.randn((2, 10000, 64), generator=g).half().to(cuda_device)
+    ids = torch.randint(0, 50, (2, 10000), generator=g).int().to(cuda_device)
+    ids[0, :9000] = 7                                   # one hot cluster
+    C = torch.randn((2, 60, 64), generator=g).to(cuda_device)   # clusters 50..59 empty
+    C_prev = C.clone()
+    _, counts, _ = km.km_update(X, ids, C, C_new=C)      # in place
+    torch.cuda.synchronize()
+    check_update(X, ids, C_prev, C, counts)
+
+
+# ------------------------------------------------------------------ fits
+
+@pytest.mark.parametrize("K", [16, 8])
+def test_fit1d_weighted_rows_per_iteration(K, cuda_device):
+    d = synth.make_workload(2, B=48, N=4096, device="cpu")
+    X, w = d["X"].to(cuda_device), d["w"].to(cuda_device)
+    C = km.km_init_grid1d(X, K)
+    C0 = C.clone()
+    iters = 30
+    _, ids, ih, ch = km.km_fit(X, C, iters, w=w, want_ids=True, want_inertia=True, want_hist=True)
+    torch.cuda.synchronize()
+    assert torch.equal(ch[0], C0) and torch.equal(ch[-1], C)
+    X64, w64 = oracle.as_f64(X.cpu()), oracle.as_f64(w.cpu())
+    hist = to_np(ch).astype(np.float64)
+    for t in range(iters):
+        Ct = hist[t]
+        ids_t, d1, d2, inertia = oracle.assign(X64, oracle.round_to_dtype(Ct, torch.float16), w64)
+        np.testing.assert_allclose(to_np(ih[t]), inertia, rtol=1e-4)
+        C_ref, _, _ = oracle.update(X64, ids_t, Ct, w64)
+        for b in range(C_ref.shape[0]):
+            err = np.linalg.norm(hist[t + 1][b] - C_ref[b]) / np.linalg.norm(C_ref[b])
+            assert err <= 1e-3, (t, b, err)
+    check_assign(X, C, ids)
+
+
+def test_fit1d_unweighted_fp32_and_worked_example(cuda_device):
+    from conftest import load_golden
+    gold = load_golden("worked_example_weight_clustering.txt")
+    vals = torch.tensor([float(v) for v in gold["values"]], dtype=torch.float32)
+    X = vals.reshape(1, -1, 1).to(cuda_device)
+    C = km.km_init_grid1d(X, 3)
+    _, ids, ih, _ = km.km_fit(X, C, 3, want_ids=True, want_inertia=True)
+    torch.cuda.synchronize()
+    got = np.sort(to_np(C)[0, :, 0])
+    printed = np.sort([float(v) for v in gold["centroids"]])
+    np.testing.assert_allclose(got, printed, atol=0.5e-4)
+    lab = to_np(ids)[0]
+    assert len(set(lab[:5])) == 1 and len(set(lab[5:10])) == 1 and lab[0] != lab[5]
+    assert to_np(ih)[1, 0] == pytest.approx(2.444e-6, rel=1e-2)
+
+
+@pytest.mark.parametrize("case", ["config1", "config3_small", "d1_generic"])
+def test_fit_generic_per_iteration(case, cuda_device):
+    if case == "config1":
+        d = synth.make_workload(1, device="cpu")
+        X, C, w = d["X"], d["C0"], None
+        iters = d["iters"]
+    elif case == "config3_small":
+        d = synth.make_workload(3, B=2, N=8192, K=256, device="cpu")
+        X, C, w = d["X"], d["C0"], None
+        iters = 3
+    else:   # d = 1 with N beyond the fused per-row kernel: the generic chain
+        d = synth.make_workload(2, B=3, N=9000, device="cpu")
+        X, w = d["X"], d["w"]
+        C = torch.from_numpy(oracle.grid_init(X, 16).astype(np.float32))
+        iters = 5
+    X, C = X.to(cuda_device), C.to(cuda_device)
+    w = None if w is None else w.to(cuda_device)
+    dtype = X.dtype
+    _, ids, ih, ch = km.km_fit(X, C, iters, w=w, want_ids=True, want_inertia=True, want_hist=True)
+    torch.cuda.synchronize()
+    X64 = oracle.as_f64(X.cpu())
+    w64 = None if w is None else oracle.as_f64(w.cpu())
+    hist = to_np(ch).astype(np.float64)
+    for t in range(iters):
+        ids_t, d1, d2, inertia = oracle.assign(X64, oracle.round_to_dtype(hist[t], dtype), w64)
+        np.testing.assert_allclose(to_np(ih[t]), inertia, rtol=1e-4)
+        C_ref, _, _ = oracle.update(X64, ids_t, hist[t], w64)
+        for b in range(C_ref.shape[0]):
+            err = np.linalg.norm(hist[t + 1][b] - C_ref[b]) / np.linalg.norm(C_ref[b])
+            assert err <= 1e-3, (t, b, err)
+    check_assign(X, C, ids)
+
+
+def test_fit_host_matches_device(cuda_device):
+    d = synth.make_workload(3, B=2, N=5000, K=200, device="cpu")
+    X, C0 = d["X"], d["C0"]
+    Xh = X.pin_memory()
+    Ch = C0.clone().pin_memory()
+    idsh = torch.empty((2, 5000), dtype=torch.int32).pin_memory()
+    inh = torch.empty((4, 2), dtype=torch.float64).pin_memory()
+    km.km_fit_host(Xh, Ch, 4, ids_host=idsh, inertia_host=inh)
+    Cd = C0.to(cuda_device)
+    _, ids, ih, _ = km.km_fit(X.to(cuda_device), Cd, 4, want_ids=True, want_inertia=True)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(Ch, Cd.cpu(), rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(inh.numpy(), to_np(ih), rtol=1e-9)
+    assert (idsh.numpy() != to_np(ids)).mean() < 1e-3
+
+
+def test_fit_k_greater_than_n_keeps_empty(cuda_device):
+    X, C = mixture(1, 50, 32, 80, torch.float16, cuda_device, seed=9)
+    C0 = C.clone()
+    _, ids, _, ch = km.km_fit(X, C, 2, want_ids=True, want_hist=True)
+    torch.cuda.synchronize()
+    assert len(set(to_np(ids)[0].tolist())) <= 50
+    # a centroid that never received a point in either iteration equals its start
+    ids0, _, _, _ = oracle.assign(oracle.as_f64(X.cpu()), oracle.round_to_dtype(C0.cpu(), torch.float16))
+    never = np.setdiff1d(np.arange(80), np.unique(ids0[0]))
+    ids1, _, _, _ = oracle.assign(oracle.as_f64(X.cpu()), oracle.round_to_dtype(ch[1].cpu(), torch.float16))
+    never = np.setdiff1d(never, np.unique(ids1[0]))
+    np.testing.assert_array_equal(to_np(C)[0, never], to_np(C0)[0, never])
