@@ -37,6 +37,7 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_STRIDE = 256;       // TMEM columns between the two accumulators
 constexpr int MAX_STAGES = 8;
 constexpr uint32_t SMEM_LIMIT = 232448;    // 227 KB opt-in per block on sm_100
+constexpr uint32_t SMEM_ATTR = SMEM_LIMIT - 1024;  // dynamic request cap (static smem is tiny)
 
 struct Layout {
     uint32_t x_off, c_off, bar_off, slot_off, merge_off, total;
@@ -57,7 +58,7 @@ __host__ __device__ inline Layout make_layout(int nkc, int bn, int stages) {
 // Largest ring depth that fits the shared-memory budget (at least 2).
 __host__ inline int pick_stages(int nkc, int bn) {
     int s = MAX_STAGES;
-    while (s > 2 && make_layout(nkc, bn, s).total + 1024u > SMEM_LIMIT) --s;
+    while (s > 2 && make_layout(nkc, bn, s).total + 1024u > SMEM_ATTR) --s;
     return s;
 }
 

@@ -273,8 +273,11 @@ km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float 
     // More than half of the shared memory per block keeps one CTA per SM, so no second CTA
     // ever waits in tcgen05.alloc for the 512 TMEM columns the first one holds.
     const size_t smem = std::max<size_t>(L.total + 1024, SMEM_LIMIT / 2 + 1024);
-    if (cudaFuncSetAttribute(assign_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
+    // The attribute is an upper bound for every later launch, so it is always set to the
+    // kernel's largest request, never to this call's size.
+    if (smem > SMEM_ATTR ||
+        cudaFuncSetAttribute(assign_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(SMEM_ATTR)) != cudaSuccess)
         return KM_ERR_CUDA;
     const int64_t items = B * p.mtiles;
     if (items > kMaxIndex) return KM_ERR_UNSUPPORTED;
@@ -364,6 +367,12 @@ km_status do_update_partial(const void *X, km_dtype dt, const int32_t *ids, cons
     using namespace km::upd;
     const bool smem_bins = K <= SMEM_K_MAX;
     const int64_t ntiles = ceil_div(N, TILE);
+    // Attributes are upper bounds for all later launches: always the kernels' largest request.
+    if (cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_K_MAX * 4) != cudaSuccess ||
+        cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (SMEM_K_MAX + TILE) * 4) != cudaSuccess)
+        return KM_ERR_CUDA;
     for (int64_t b0 = 0; b0 < B; b0 += kMaxGridY) {
         const int64_t nb = std::min<int64_t>(kMaxGridY, B - b0);
         dim3 grid(static_cast<unsigned>(ntiles), static_cast<unsigned>(nb));
@@ -375,12 +384,6 @@ km_status do_update_partial(const void *X, km_dtype dt, const int32_t *ids, cons
                                                                       u.offsets, u.cursor);
     if (launch_status() != KM_OK) return KM_ERR_CUDA;
     const size_t scatter_smem = smem_bins ? static_cast<size_t>(K + TILE) * 4 : 0;
-    if (smem_bins && cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          static_cast<int>(scatter_smem)) != cudaSuccess)
-        return KM_ERR_CUDA;
-    if (smem_bins && cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          static_cast<int>(K * 4)) != cudaSuccess)
-        return KM_ERR_CUDA;
     for (int64_t b0 = 0; b0 < B; b0 += kMaxGridY) {
         const int64_t nb = std::min<int64_t>(kMaxGridY, B - b0);
         dim3 grid(static_cast<unsigned>(ntiles), static_cast<unsigned>(nb));
@@ -404,7 +407,7 @@ km_status run_fit1d(const void *X, const float *w, int64_t B, int64_t N, int64_t
     while (NP < N) NP <<= 1;
     const size_t smem = static_cast<size_t>(NP) * 12;
     if (cudaFuncSetAttribute(km::fit1d::fit1d_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
+                             km::fit1d::NMAX * 12) != cudaSuccess)
         return KM_ERR_CUDA;
     km::fit1d::fit1d_kernel<T><<<static_cast<unsigned>(B), km::fit1d::THREADS, smem, st>>>(
         static_cast<const T *>(X), w, static_cast<int>(B), static_cast<int>(N), NP,

@@ -93,7 +93,10 @@ km_status km_prep(const float *C, km_dtype dtype, int64_t B, int64_t K, int64_t 
  *   chosen centroid, max(0, .); inertia[B] fp64 out or NULL: sum_i w_i * mind_i.
  * fp16/bf16 with d % 8 == 0, 8 <= d <= 256 and 16-byte aligned X/Cx run on the tcgen05 tensor
  * cores (fp32 accumulation of <x,c>); every other case runs an exact-fp32 CUDA-core kernel that
- * evaluates sum_j (x_j - c_j)^2 directly.
+ * evaluates sum_j (x_j - c_j)^2 directly. On the tensor-core path mind is formed as
+ * ||x||^2 + (||c||^2 - 2<x,c>) in fp32, so its absolute error is a small multiple of
+ * 2^-24 (||x||^2 + ||c||^2); for points almost on their centroid that can exceed 1e-4 of the
+ * distance itself (the assignment is unaffected except at near-ties).
  */
 km_status km_assign(const void *X, km_dtype dtype, const void *Cx, const float *cn,
                     const float *w, int64_t B, int64_t N, int64_t K, int64_t d, int32_t *ids,

@@ -86,8 +86,8 @@ def check_update(X, ids_gpu, C_prev, C_new_gpu, counts_gpu, *, w=None, wsum_gpu=
     return C_ref
 
 
-def mixture(B, N, d, K, dtype, device, seed=0, sigma=0.3):
-    """Clustered points plus K initial centroids drawn among them (plus a little noise)."""
+def mixture(B, N, d, K, dtype, device, seed=0, sigma=0.3, c_noise=0.3):
+    """Clustered points plus K initial centroids drawn among them (plus ``c_noise`` noise)."""
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     ncomp = max(1, min(K, 64))
@@ -96,5 +96,5 @@ def mixture(B, N, d, K, dtype, device, seed=0, sigma=0.3):
     X = torch.gather(mu, 1, comp[..., None].expand(B, N, d)) + sigma * torch.randn((B, N, d), generator=g)
     idx = torch.stack([torch.randperm(N, generator=g)[:K] if K <= N else torch.randint(0, N, (K,), generator=g)
                        for _ in range(B)])
-    C = torch.gather(X, 1, idx[..., None].expand(B, K, d)) + 0.05 * torch.randn((B, K, d), generator=g)
+    C = torch.gather(X, 1, idx[..., None].expand(B, K, d)) + c_noise * torch.randn((B, K, d), generator=g)
     return X.to(dtype).to(device), C.float().to(device)
