@@ -61,6 +61,8 @@ def _load():
         "km_fit_host": ([P, I, P, I64, I64, I64, I64, P, I, P, P, P, SZ, P], I),
         "km_device_error": ([P, ctypes.POINTER(I)], I),
         "km_assign_uses_tensor_cores": ([I, I64, P, P], I),
+        "km_update_noalloc": ([P, I, P, P, I64, I64, I64, I64, P, P, P, P, P], I),
+        "km_noalloc_scratch_needed": ([I64, I64, I64, I64], SZ),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)

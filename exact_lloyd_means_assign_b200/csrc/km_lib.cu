@@ -645,3 +645,59 @@ km_status km_device_error(void *stream, int *code) {
 }
 
 }  // extern "C"
+
+// =================================================================== allocation-free update
+//
+// Scratch for km_update_noalloc: one file-scope device array, present on every device that
+// loads the library until the process exits. Host code must not hand the array's name to a
+// kernel (on the host it only names a stand-in); its device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+static __device__ __align__(256) uint8_t g_km_noalloc_scratch[KM_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+void *noalloc_scratch_device_ptr() {
+    static void *cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!cache[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_km_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+        cache[dev] = p;
+    }
+    return cache[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t km_noalloc_scratch_needed(int64_t B, int64_t N, int64_t K, int64_t d) {
+    if (!sizes_ok(B, N, K, d)) return 0;
+    Carver c(nullptr);
+    carve_update(c, B, N, K, d);
+    return c.off;
+}
+
+km_status km_update_noalloc(const void *X, km_dtype dtype, const int32_t *ids, const float *w,
+                            int64_t B, int64_t N, int64_t K, int64_t d, const float *C_prev,
+                            float *C_new, int32_t *counts, float *wsum, void *stream) {
+    if (!X || !ids || !C_prev || !C_new || !counts || !valid_dtype(dtype) || !sizes_ok(B, N, K, d) ||
+        !elem_aligned(X, dtype) || !aligned(ids, 4) || !aligned(counts, 4) || !aligned(C_prev, 4) ||
+        !aligned(C_new, 4) || (w && !aligned(w, 4)) || (wsum && !aligned(wsum, 4)))
+        return KM_ERR_INVALID_ARG;
+    if (km_noalloc_scratch_needed(B, N, K, d) > KM_NOALLOC_SCRATCH_BYTES) return KM_ERR_WORKSPACE;
+    void *scratch = noalloc_scratch_device_ptr();
+    if (!scratch) return KM_ERR_CUDA;
+    Carver r(scratch);
+    UpdateWs u = carve_update(r, B, N, K, d);
+    float *ws_w = wsum ? wsum : (w ? u.wsum : nullptr);
+    // do_update_partial clears counts, sums and wsum first, so the previous call's contents of
+    // the shared array never leak into this one.
+    km_status s = do_update_partial(X, dtype, ids, w, B, N, K, d, u.sums, ws_w, counts, u, S(stream));
+    if (s != KM_OK) return s;
+    return finalize_dispatch(u.sums, w ? ws_w : nullptr, counts, C_prev, B * K, d, C_new, KM_F32,
+                             nullptr, nullptr, S(stream));
+}
+
+}  // extern "C"

@@ -187,6 +187,32 @@ km_status km_fit_host(const void *X_host, km_dtype dtype, const float *w_host, i
  */
 km_status km_device_error(void *stream, int *code);
 
+/*
+ * km_update for callers that cannot allocate device memory: the same computation and outputs
+ * as km_update, but the scratch (offsets, cursors, permutation, partial sums) lives in one
+ * array of the library itself, KM_NOALLOC_SCRATCH_BYTES (32 MiB) per device, reserved when the
+ * library is loaded and held until the process exits. No page text has a counterpart: this is
+ * an interface convenience, not part of the method.
+ * Meant for code that must not call cudaMalloc/cudaFree at that point (the allocation calls
+ * can synchronise the device and stall other streams, and some embeddings hand the library no
+ * allocator at all), so there is no workspace to pass.
+ *   - Sizes whose scratch exceeds the array (see km_noalloc_scratch_needed) are rejected with
+ *     KM_ERR_WORKSPACE before anything is enqueued.
+ *   - The first call on a device looks up the array's device address with
+ *     cudaGetSymbolAddress (once per device, on the current device); make that first call
+ *     before any stream capture.
+ *   - Every call uses the same array: calls that can overlap on the GPU (different streams,
+ *     or several host threads) race with each other and must be serialised by the caller.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ */
+#define KM_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+km_status km_update_noalloc(const void *X, km_dtype dtype, const int32_t *ids, const float *w,
+                            int64_t B, int64_t N, int64_t K, int64_t d, const float *C_prev,
+                            float *C_new, int32_t *counts, float *wsum, void *stream);
+
+/* Bytes of the static scratch km_update_noalloc needs for these sizes (0 on invalid sizes). */
+size_t km_noalloc_scratch_needed(int64_t B, int64_t N, int64_t K, int64_t d);
+
 #ifdef __cplusplus
 }
 #endif
