@@ -4,8 +4,10 @@
 // finalize: C_new = sums / wsum for non-empty clusters, else C_prev (the mean S_j / N_j of the
 //           Lloyd recap in the steinslab e-means daily); optionally also Cx and cn for the next
 //           assignment, so a multi-iteration fit never runs prep twice.
-// cnpad:    the norm row the tensor-core assignment reads, padded to whole centroid tiles with
-//           +inf so padding columns can never win the argmin.
+// caug:     the extra reduction step the tensor-core assignment appends to every centroid tile:
+//           per centroid 16 bf16 values [1, a, b, c, 0...] with a + b + c = ||c||^2 / 2 (a
+//           three-piece bf16 split, exact to about 2^-27 relative), padded to whole tiles with
+//           [0, 1e30, 0...] rows so padding columns can never win the argmin.
 #pragma once
 
 #include "km_common.cuh"
@@ -60,30 +62,45 @@ __global__ void finalize_kernel(const float *__restrict__ sums, const float *__r
     }
 }
 
-// cnp[b, k] for k < Kp: ||Cx[b,k]||^2 (from `cn` when given, else computed from Cx) for k < K,
-// +inf for the padding k >= K. One warp per (b, k).
+// caug[b, k, 0..15] (bf16) for k < Kp, one warp per (b, k). ||Cx[b,k]||^2 comes from `cn` when
+// given, else it is computed from Cx.
 template <typename T>
-__global__ void cnpad_kernel(const T *__restrict__ Cx, const float *__restrict__ cn, int B, int K,
-                             int Kp, int d, float *__restrict__ cnp) {
+__global__ void caug_kernel(const T *__restrict__ Cx, const float *__restrict__ cn, int B, int K,
+                            int Kp, int d, __nv_bfloat16 *__restrict__ caug) {
     const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= static_cast<int64_t>(B) * Kp) return;
     const int b = static_cast<int>(row / Kp), k = static_cast<int>(row % Kp);
-    float v;
-    if (k >= K) {
-        v = INFINITY;
-    } else if (cn) {
-        v = cn[static_cast<int64_t>(b) * K + k];
-    } else {
-        const T *c = Cx + (static_cast<int64_t>(b) * K + k) * d;
-        float s = 0.f;
-        for (int j = lane; j < d; j += 32) {
-            const float f = Cvt<T>::to_f(c[j]);
-            s = fmaf(f, f, s);
+    float v = 0.f;
+    if (k < K) {
+        if (cn) {
+            v = cn[static_cast<int64_t>(b) * K + k];
+        } else {
+            const T *c = Cx + (static_cast<int64_t>(b) * K + k) * d;
+            float s = 0.f;
+            for (int j = lane; j < d; j += 32) {
+                const float f = Cvt<T>::to_f(c[j]);
+                s = fmaf(f, f, s);
+            }
+            v = warp_sum(s);
         }
-        v = warp_sum(s);
     }
-    if (lane == 0) cnp[row] = v;
+    // Row layout [1, 1, a, b, c, 0 x 11]: the point side is [x1, x2, 1, 1, 1, 0 x 11], so the
+    // extra reduction step adds x1 + x2 + a + b + c = ||x||^2/2 (split) + ||c||^2/2.
+    if (lane < 16) {
+        float e = 0.f;
+        if (k >= K) {
+            e = (lane == 2) ? 1e30f : 0.f;
+        } else {
+            const float h = 0.5f * v;
+            const float a = __bfloat162float(__float2bfloat16_rn(h));
+            const float r1 = h - a;
+            const float b2 = __bfloat162float(__float2bfloat16_rn(r1));
+            const float c3 = r1 - b2;
+            e = lane < 2 ? 1.f : lane == 2 ? a : lane == 3 ? b2 : lane == 4 ? c3 : 0.f;
+        }
+        caug[row * 16 + lane] = __float2bfloat16_rn(e);
+    }
 }
 
 }  // namespace km

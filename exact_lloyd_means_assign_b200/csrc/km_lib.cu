@@ -62,7 +62,7 @@ inline int tc_bn(int64_t K) { return K > 128 ? 256 : (K > 64 ? 128 : 64); }
 inline int64_t tc_kp(int64_t K) { return ceil_div(K, tc_bn(K)) * tc_bn(K); }
 
 inline size_t ws_assign(int64_t B, int64_t K, int64_t d, km_dtype dt) {
-    return tc_shape_ok(dt, d) ? align_up(static_cast<size_t>(B * tc_kp(K)) * 4) : 0;
+    return tc_shape_ok(dt, d) ? align_up(static_cast<size_t>(B * tc_kp(K)) * 32) : 0;
 }
 
 struct UpdateWs {
@@ -212,25 +212,47 @@ km_status run_assign_simt(const void *X, const void *Cx, const float *w, int64_t
     return KM_OK;
 }
 
+template <typename T, int BN>
+km_status launch_assign_tc(const CUtensorMap &tmX, const CUtensorMap &tmC, const CUtensorMap &tmA,
+                           km::tc::Params &p, int64_t items, cudaStream_t st) {
+    using namespace km::tc;
+    p.stages = pick_stages(p.nkc, BN);
+    const Layout L = make_layout(p.nkc, BN, p.stages);
+    // More than half of the shared memory per block keeps one CTA per SM, so no second CTA
+    // ever waits in tcgen05.alloc for the 512 TMEM columns the first one holds.
+    const size_t smem = std::max<size_t>(L.total + 1024, SMEM_LIMIT / 2 + 1024);
+    // The attribute is an upper bound for every later launch, so it is always set to the
+    // kernel's largest request, never to this call's size.
+    if (smem > SMEM_ATTR ||
+        cudaFuncSetAttribute(assign_tc_kernel<T, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(SMEM_ATTR)) != cudaSuccess)
+        return KM_ERR_CUDA;
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(items, num_sms()));
+    assign_tc_kernel<T, BN><<<grid, NUM_THREADS, smem, st>>>(tmX, tmC, tmA, p);
+    return launch_status();
+}
+
+// `caug` (workspace) holds B * tc_kp(K) rows of 16 bf16: the centroid side of the extra
+// reduction step that adds ||c||^2 / 2 (see km_assign_tc.cuh).
 template <typename T>
 km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float *cn,
                         const float *w, int64_t B, int64_t N, int64_t K, int64_t d, int32_t *ids,
-                        float *mind, double *inertia, float *cnp, cudaStream_t st) {
+                        float *mind, double *inertia, void *caug, cudaStream_t st) {
     using namespace km::tc;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return KM_ERR_CUDA;
     const int bn = tc_bn(K);
     const int64_t Kp = tc_kp(K);
     const int nkc = static_cast<int>(ceil_div(d, KC));
-    km::cnpad_kernel<T><<<static_cast<unsigned>(ceil_div(B * Kp, 8)), 256, 0, st>>>(
+    km::caug_kernel<T><<<static_cast<unsigned>(ceil_div(B * Kp, 8)), 256, 0, st>>>(
         static_cast<const T *>(Cx), cn, static_cast<int>(B), static_cast<int>(K),
-        static_cast<int>(Kp), static_cast<int>(d), cnp);
+        static_cast<int>(Kp), static_cast<int>(d), static_cast<__nv_bfloat16 *>(caug));
     if (launch_status() != KM_OK) return KM_ERR_CUDA;
 
     const CUtensorMapDataType tdt =
         dt == KM_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const cuuint32_t estr[3] = {1, 1, 1};
-    CUtensorMap tmX, tmC;
+    CUtensorMap tmX, tmC, tmA;
     {
         const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                                     static_cast<cuuint64_t>(B)};
@@ -251,53 +273,54 @@ km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float 
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return KM_ERR_CUDA;
     }
+    {
+        const cuuint64_t dims[3] = {16, static_cast<cuuint64_t>(Kp), static_cast<cuuint64_t>(B)};
+        const cuuint64_t strides[2] = {32, static_cast<cuuint64_t>(Kp * 32)};
+        const cuuint32_t box[3] = {16, static_cast<cuuint32_t>(bn), 1};
+        if (enc(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, caug, dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return KM_ERR_CUDA;
+    }
     Params p;
     p.B = static_cast<int>(B);
     p.N = static_cast<int>(N);
     p.K = static_cast<int>(K);
     p.d = static_cast<int>(d);
     p.nkc = nkc;
-    p.bn = bn;
     p.nct = static_cast<int>(Kp / bn);
     p.mtiles = static_cast<int>(ceil_div(N, BM));
-    p.stages = pick_stages(nkc, bn);
-    p.need_xn = (mind || inertia) ? 1 : 0;
-    p.idesc = km::mma_idesc_f16(dt == KM_BF16 ? 1u : 0u, BM, static_cast<uint32_t>(bn));
-    p.cnp = cnp;
-    p.Kp = static_cast<int>(Kp);
+    p.stages = 2;
+    p.need_dist = (mind || inertia) ? 1 : 0;
+    // main step: A (the points) negated, so the accumulator collects -<x, c>
+    p.idesc_main = km::mma_idesc_f16(dt == KM_BF16 ? 1u : 0u, BM, static_cast<uint32_t>(bn)) | (1u << 13);
+    p.idesc_aug = km::mma_idesc_f16(1u, BM, static_cast<uint32_t>(bn));
     p.w = w;
     p.ids = ids;
     p.mind = mind;
     p.inertia = inertia;
-    const Layout L = make_layout(nkc, bn, p.stages);
-    // More than half of the shared memory per block keeps one CTA per SM, so no second CTA
-    // ever waits in tcgen05.alloc for the 512 TMEM columns the first one holds.
-    const size_t smem = std::max<size_t>(L.total + 1024, SMEM_LIMIT / 2 + 1024);
-    // The attribute is an upper bound for every later launch, so it is always set to the
-    // kernel's largest request, never to this call's size.
-    if (smem > SMEM_ATTR ||
-        cudaFuncSetAttribute(assign_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(SMEM_ATTR)) != cudaSuccess)
-        return KM_ERR_CUDA;
     const int64_t items = B * p.mtiles;
     if (items > kMaxIndex) return KM_ERR_UNSUPPORTED;
-    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(items, num_sms()));
-    assign_tc_kernel<T><<<grid, NUM_THREADS, smem, st>>>(tmX, tmC, p);
-    return launch_status();
+    switch (bn) {
+        case 64: return launch_assign_tc<T, 64>(tmX, tmC, tmA, p, items, st);
+        case 128: return launch_assign_tc<T, 128>(tmX, tmC, tmA, p, items, st);
+        default: return launch_assign_tc<T, 256>(tmX, tmC, tmA, p, items, st);
+    }
 }
 
-// Validated-argument assignment; `cnp` must hold B * tc_kp(K) floats when the TC path can run.
+// Validated-argument assignment; `caug` must hold ws_assign(B, K, d) bytes when the tensor-core
+// path can run.
 km_status do_assign(const void *X, km_dtype dt, const void *Cx, const float *cn, const float *w,
                     int64_t B, int64_t N, int64_t K, int64_t d, int32_t *ids, float *mind,
-                    double *inertia, float *cnp, cudaStream_t st) {
+                    double *inertia, void *caug, cudaStream_t st) {
     if (inertia && cudaMemsetAsync(inertia, 0, static_cast<size_t>(B) * 8, st) != cudaSuccess)
         return KM_ERR_CUDA;
-    const bool tc = tc_shape_ok(dt, d) && aligned(X, 16) && aligned(Cx, 16) && cnp != nullptr &&
+    const bool tc = tc_shape_ok(dt, d) && aligned(X, 16) && aligned(Cx, 16) && caug != nullptr &&
                     B * ceil_div(N, 128) <= kMaxIndex;
     if (tc) {
         if (dt == KM_F16)
-            return run_assign_tc<__half>(X, dt, Cx, cn, w, B, N, K, d, ids, mind, inertia, cnp, st);
-        return run_assign_tc<__nv_bfloat16>(X, dt, Cx, cn, w, B, N, K, d, ids, mind, inertia, cnp, st);
+            return run_assign_tc<__half>(X, dt, Cx, cn, w, B, N, K, d, ids, mind, inertia, caug, st);
+        return run_assign_tc<__nv_bfloat16>(X, dt, Cx, cn, w, B, N, K, d, ids, mind, inertia, caug, st);
     }
     switch (dt) {
         case KM_F32: return run_assign_simt<float>(X, Cx, w, B, N, K, d, ids, mind, inertia, st);
@@ -434,7 +457,7 @@ km_status do_fit(const void *X, km_dtype dt, const float *w, int64_t B, int64_t 
     FitWs f = carve_fit(c, B, N, K, d, dt);
     Carver r(f.rest);
     UpdateWs u = carve_update(r, B, N, K, d);
-    float *cnp = static_cast<float *>(f.rest);  // assignment scratch shares the update region
+    void *caug = f.rest;  // assignment scratch shares the update region (used one after the other)
     const size_t cbytes = static_cast<size_t>(B * K * d) * 4;
     km_status s = prep_dispatch(C, dt, B * K, d, f.Cx, f.cn, st);
     if (s != KM_OK) return s;
@@ -443,7 +466,7 @@ km_status do_fit(const void *X, km_dtype dt, const float *w, int64_t B, int64_t 
                                       cudaMemcpyDeviceToDevice, st) != cudaSuccess)
             return KM_ERR_CUDA;
         double *in = inertia_hist ? inertia_hist + static_cast<int64_t>(t) * B : nullptr;
-        s = do_assign(X, dt, f.Cx, f.cn, w, B, N, K, d, f.ids, nullptr, in, cnp, st);
+        s = do_assign(X, dt, f.Cx, f.cn, w, B, N, K, d, f.ids, nullptr, in, caug, st);
         if (s != KM_OK) return s;
         s = do_update_partial(X, dt, f.ids, w, B, N, K, d, u.sums, w ? u.wsum : nullptr, f.counts, u, st);
         if (s != KM_OK) return s;
@@ -453,7 +476,7 @@ km_status do_fit(const void *X, km_dtype dt, const float *w, int64_t B, int64_t 
     if (C_hist && cudaMemcpyAsync(C_hist + static_cast<int64_t>(iters) * B * K * d, C, cbytes,
                                   cudaMemcpyDeviceToDevice, st) != cudaSuccess)
         return KM_ERR_CUDA;
-    if (ids) return do_assign(X, dt, f.Cx, f.cn, w, B, N, K, d, ids, nullptr, nullptr, cnp, st);
+    if (ids) return do_assign(X, dt, f.Cx, f.cn, w, B, N, K, d, ids, nullptr, nullptr, caug, st);
     return KM_OK;
 }
 
@@ -514,8 +537,8 @@ km_status km_assign(const void *X, km_dtype dtype, const void *Cx, const float *
         return KM_ERR_INVALID_ARG;
     const size_t need = ws_assign(B, K, d, dtype);
     if (need && (!ws || ws_bytes < need || !aligned(ws, kAlign))) return KM_ERR_WORKSPACE;
-    return do_assign(X, dtype, Cx, cn, w, B, N, K, d, ids, mind, inertia,
-                     need ? static_cast<float *>(ws) : nullptr, S(stream));
+    return do_assign(X, dtype, Cx, cn, w, B, N, K, d, ids, mind, inertia, need ? ws : nullptr,
+                     S(stream));
 }
 
 km_status km_update_partial(const void *X, km_dtype dtype, const int32_t *ids, const float *w,

@@ -56,11 +56,11 @@ def test_status_strings_and_version(lib):
 
 def test_workspace_sizes(lib):
     f16, f32 = torch.float16, torch.float32
-    # the exact-fp32 CUDA-core assignment needs no workspace; the tensor-core one needs the
-    # padded norm row: B * ceil(K/256)*256 floats
+    # the exact-fp32 CUDA-core assignment needs no workspace; the tensor-core one needs one
+    # 16-value bf16 augmentation row per (padded) centroid: B * ceil(K/bn)*bn * 32 bytes
     assert km.km_workspace_size(km.KM_OP_ASSIGN, 2, 100, 32, 16, f32) == 0
-    assert km.km_workspace_size(km.KM_OP_ASSIGN, 2, 100, 300, 128, f16) == 2 * 512 * 4
-    assert km.km_workspace_size(km.KM_OP_ASSIGN, 1, 100, 50, 128, f16) == 256
+    assert km.km_workspace_size(km.KM_OP_ASSIGN, 2, 100, 300, 128, f16) == 2 * 512 * 32
+    assert km.km_workspace_size(km.KM_OP_ASSIGN, 1, 100, 50, 128, f16) == 64 * 32
     up = km.km_workspace_size(km.KM_OP_UPDATE, 32, 65536, 1024, 128, f16)
     assert up >= 32 * 65536 * 4 + 32 * 1024 * 128 * 4
     fit = km.km_workspace_size(km.KM_OP_FIT, 32, 65536, 1024, 128, f16)
