@@ -58,11 +58,18 @@ struct Carver {
 inline bool tc_shape_ok(km_dtype dt, int64_t d) {
     return dt != KM_F32 && d % 8 == 0 && d >= 8 && d <= 256;
 }
-inline int tc_bn(int64_t K) { return K > 128 ? 256 : (K > 64 ? 128 : 64); }
-inline int64_t tc_kp(int64_t K) { return ceil_div(K, tc_bn(K)) * tc_bn(K); }
+// Centroids per SM-pair tile: the smallest of 64/128/256 that covers K, narrowed while the
+// point tile plus two ring stages would not fit in shared memory (large d).
+inline int tc_bn(int64_t K, int64_t d) {
+    int bn = K > 128 ? 256 : (K > 64 ? 128 : 64);
+    const int nkc = static_cast<int>(ceil_div(d, km::tc::KC));
+    while (bn > 64 && km::tc::pick_stages(nkc, bn) == 0) bn /= 2;
+    return bn;
+}
+inline int64_t tc_kp(int64_t K, int64_t d) { return ceil_div(K, tc_bn(K, d)) * tc_bn(K, d); }
 
 inline size_t ws_assign(int64_t B, int64_t K, int64_t d, km_dtype dt) {
-    return tc_shape_ok(dt, d) ? align_up(static_cast<size_t>(B * tc_kp(K)) * 32) : 0;
+    return tc_shape_ok(dt, d) ? align_up(static_cast<size_t>(B * tc_kp(K, d)) * 32) : 0;
 }
 
 struct UpdateWs {
@@ -217,6 +224,7 @@ km_status launch_assign_tc(const CUtensorMap &tmX, const CUtensorMap &tmC, const
                            km::tc::Params &p, int64_t items, cudaStream_t st) {
     using namespace km::tc;
     p.stages = pick_stages(p.nkc, BN);
+    if (p.stages < 2) return KM_ERR_UNSUPPORTED;
     const Layout L = make_layout(p.nkc, BN, p.stages);
     // More than half of the shared memory per block keeps one CTA per SM, so no second CTA
     // ever waits in tcgen05.alloc for the 512 TMEM columns the first one holds.
@@ -227,7 +235,33 @@ km_status launch_assign_tc(const CUtensorMap &tmX, const CUtensorMap &tmC, const
         cudaFuncSetAttribute(assign_tc_kernel<T, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(SMEM_ATTR)) != cudaSuccess)
         return KM_ERR_CUDA;
-    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(items, num_sms()));
+    // Persistent clusters (SM pairs): as many as can be resident at once (a pair needs two SMs
+    // of one GPC, so this can be below half the SM count), never more than the work items.
+    static int resident[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int max_clusters = (dev >= 0 && dev < 64) ? resident[dev] : 0;
+    if (max_clusters <= 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(2 * std::max(1, num_sms() / 2)));
+        cfg.blockDim = dim3(NUM_THREADS);
+        cfg.dynamicSmemBytes = SMEM_ATTR;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = 2;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&max_clusters, assign_tc_kernel<T, BN>, &cfg) != cudaSuccess ||
+            max_clusters <= 0) {
+            cudaGetLastError();
+            max_clusters = std::max(1, num_sms() / 2);
+        }
+        if (dev >= 0 && dev < 64) resident[dev] = max_clusters;
+    }
+    const int64_t clusters = std::min<int64_t>(items, max_clusters);
+    const unsigned grid = static_cast<unsigned>(2 * clusters);
     assign_tc_kernel<T, BN><<<grid, NUM_THREADS, smem, st>>>(tmX, tmC, tmA, p);
     return launch_status();
 }
@@ -241,8 +275,8 @@ km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float 
     using namespace km::tc;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return KM_ERR_CUDA;
-    const int bn = tc_bn(K);
-    const int64_t Kp = tc_kp(K);
+    const int bn = tc_bn(K, d);
+    const int64_t Kp = tc_kp(K, d);
     const int nkc = static_cast<int>(ceil_div(d, KC));
     km::caug_kernel<T><<<static_cast<unsigned>(ceil_div(B * Kp, 8)), 256, 0, st>>>(
         static_cast<const T *>(Cx), cn, static_cast<int>(B), static_cast<int>(K),
@@ -267,7 +301,8 @@ km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float 
         const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(K),
                                     static_cast<cuuint64_t>(B)};
         const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(K * d * 2)};
-        const cuuint32_t box[3] = {static_cast<cuuint32_t>(KC), static_cast<cuuint32_t>(bn), 1};
+        // each CTA of a pair stages half of every centroid tile
+        const cuuint32_t box[3] = {static_cast<cuuint32_t>(KC), static_cast<cuuint32_t>(bn / 2), 1};
         if (enc(&tmC, tdt, 3, const_cast<void *>(Cx), dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -276,7 +311,7 @@ km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float 
     {
         const cuuint64_t dims[3] = {16, static_cast<cuuint64_t>(Kp), static_cast<cuuint64_t>(B)};
         const cuuint64_t strides[2] = {32, static_cast<cuuint64_t>(Kp * 32)};
-        const cuuint32_t box[3] = {16, static_cast<cuuint32_t>(bn), 1};
+        const cuuint32_t box[3] = {16, static_cast<cuuint32_t>(bn / 2), 1};
         if (enc(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, caug, dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -289,12 +324,14 @@ km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float 
     p.d = static_cast<int>(d);
     p.nkc = nkc;
     p.nct = static_cast<int>(Kp / bn);
-    p.mtiles = static_cast<int>(ceil_div(N, BM));
+    p.mtiles = static_cast<int>(ceil_div(N, 2 * BM));   // 256-point items, one per SM pair
     p.stages = 2;
     p.need_dist = (mind || inertia) ? 1 : 0;
-    // main step: A (the points) negated, so the accumulator collects -<x, c>
-    p.idesc_main = km::mma_idesc_f16(dt == KM_BF16 ? 1u : 0u, BM, static_cast<uint32_t>(bn)) | (1u << 13);
-    p.idesc_aug = km::mma_idesc_f16(1u, BM, static_cast<uint32_t>(bn));
+    // M = 256 across the pair; main step with A (the points) negated, so the accumulator
+    // collects -<x, c>
+    p.idesc_main =
+        km::mma_idesc_f16(dt == KM_BF16 ? 1u : 0u, 2 * BM, static_cast<uint32_t>(bn)) | (1u << 13);
+    p.idesc_aug = km::mma_idesc_f16(1u, 2 * BM, static_cast<uint32_t>(bn));
     p.w = w;
     p.ids = ids;
     p.mind = mind;
