@@ -17,10 +17,10 @@
 // 2^-27 relative. Padding centroids carry 1e30 so they never win.
 //
 // Because the accumulator is (half) the distance itself, the epilogue keeps the argmin as a
-// packed key: the low 5 mantissa bits are replaced by the column index within a 32-column chunk,
-// and one three-input float min per two columns keeps both the minimum and its position (equal
-// keys resolve to the lower index; values closer than 2^-18 relative resolve by index, far inside
-// the near-tie band). Per score: one LOP3 and half a FMNMX.
+// packed key: the low log2(W) mantissa bits (W = columns one warp reads per tile, at most 64)
+// are replaced by the column index, and one three-input float min per two columns keeps both
+// the minimum and its position (equal keys resolve to the lower index; values closer than 2^-17
+// relative resolve by index, far inside the near-tie band). Per score: one LOP3 and half a FMNMX.
 //
 // SM pairs. A cluster of two CTAs runs one tcgen05.mma.cta_group::2 per K step: M = 256 points
 // (128 per CTA, each CTA's rows in its own shared memory and its own TMEM lanes) by N = bn
@@ -29,23 +29,29 @@
 // owns the "full" barriers; both CTAs' centroid loads complete on them (2-SM TMA form), and MMA
 // completion is committed to both CTAs' barriers (multicast commit). No TMA load uses multicast.
 //
-// Keeping the tensor pipe fed. The MMA queue is shallow, so the issuing thread must not spend
-// long between tiles: one ring stage holds a whole centroid tile (all K chunks plus its
-// augmentation rows) behind one barrier, so a tile costs the MMA thread two barrier checks
-// (accumulator free, operands landed; the first probe is non-blocking) and two commits around
-// its MMAs, with descriptors formed by adding offsets to precomputed words. Point tiles come from
-// their own producer warp, so the centroid stream never waits behind the epilogue.
+// Keeping the tensor pipe fed. The MMA queue holds only a couple of instructions, so whatever
+// the issuing warp does between the last MMA of one tile and the first of the next is a bubble.
+// That gap is kept to one commit: a ring stage holds a whole centroid tile behind one barrier,
+// the stage and the point buffer are handed back by the epilogue (which has seen the tile's
+// completion) rather than by further commits, and the next tile's barriers are probed while the
+// current tile's MMAs are still queued. The MMA warp runs converged and issues from one elected
+// lane, so its addresses and descriptors stay warp-uniform.
 //
-// Roles per CTA (persistent clusters, 15 warps):
-//   warp 0    centroid producer: own half of each centroid tile [bn/2 x d] and its augmentation
-//             rows [bn/2 x 16] into one stage of a ring (L2 evict-last: every CTA re-reads them).
-//   warp 1    TMEM allocation (512 columns, both CTAs); in the leader also the MMA issuer.
-//   warps 2-9 epilogue: TMEM lane quarter = warp % 4, column half = (warp - 2) / 4; one point
-//             row per thread; TMEM loads pipelined one chunk ahead; accumulator released as soon
-//             as its last chunk is in registers.
-//   warps 10-13 norms: ||x||^2 of the point tile as soon as it lands and the point-side
-//             augmentation row, so the MMA never waits for the epilogue between work items.
-//   warp 14   point producer: own point tile [128 x d], double-buffered (L2 evict-first).
+// Keeping the epilogue off the critical path. TMEM loads have a long latency, so each epilogue
+// warp issues all of its columns of a tile at once (one wait per tile) and sixteen warps share
+// the accumulator: four TMEM lane quarters x four column quarters. The accumulator is released
+// as soon as the registers hold it; the min/argmin math runs while the next tile is computed.
+//
+// Roles per CTA (persistent clusters, 20 warps: five per SM sub-partition, which leaves 96
+// registers per thread):
+//   warp 0      centroid producer: own half of each centroid tile [bn/2 x d] and its augmentation
+//               rows [bn/2 x 16] into one stage of a ring (L2 evict-last: every CTA re-reads them).
+//   warp 1      TMEM allocation (512 columns, both CTAs); in the leader also the MMA issuer.
+//   warp 2      point producer: own point tile [128 x d], double-buffered (L2 evict-first).
+//   warp 3      norms: ||x||^2 of the point tile as soon as it lands, the point-side augmentation
+//               rows and delta, so the MMA never waits for the epilogue between work items.
+//   warps 4-19  epilogue: TMEM lane quarter = warp % 4, column quarter = (warp - 4) / 4; one point
+//               row per thread.
 //
 // All mbarrier waits are bounded (km_common.cuh). On a timeout every role leaves its loop, the
 // producers wait for the copies they issued, the leader drains its MMAs, the pair synchronises
@@ -61,19 +67,20 @@ constexpr int BM = 128;                     // points per CTA (TMEM lanes); 256 
 constexpr int KC = 64;                      // 16-bit elements per 128-byte swizzle row
 constexpr uint32_t XCHUNK = BM * 128;       // bytes of one [128 x 64] point chunk
 constexpr uint32_t XAUG_BYTES = BM * 32;    // [128 x 16] bf16 point-side augmentation
-constexpr int NUM_EPI_WARPS = 8;
-constexpr int NUM_NORM_WARPS = 4;
+constexpr int NUM_EPI_WARPS = 16;
+constexpr int NUM_NORM_WARPS = 1;
 constexpr int WARP_CPROD = 0;
 constexpr int WARP_MMA = 1;
-constexpr int WARP_EPI0 = 2;
-constexpr int WARP_NORM0 = 10;
-constexpr int WARP_XPROD = 14;
-constexpr int NUM_THREADS = 32 * 15;
+constexpr int WARP_XPROD = 2;
+constexpr int WARP_NORM0 = 3;
+constexpr int WARP_EPI0 = WARP_NORM0 + NUM_NORM_WARPS;
+constexpr int NUM_THREADS = 32 * (WARP_EPI0 + NUM_EPI_WARPS);
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_STRIDE = 256;        // TMEM columns between the two accumulators
 constexpr int MAX_STAGES = 8;
 constexpr uint32_t SMEM_LIMIT = 232448;     // 227 KB opt-in per block on sm_100
 constexpr uint32_t SMEM_ATTR = SMEM_LIMIT - 1024;  // dynamic request cap (static smem is tiny)
+constexpr int NUM_BARS_FIXED = 13;
 
 // Bytes one CTA stages per centroid tile: nkc chunks of [bn/2 x 64] plus [bn/2 x 16] bf16.
 __host__ __device__ inline uint32_t cstage_bytes(int nkc, int bn) {
@@ -81,7 +88,7 @@ __host__ __device__ inline uint32_t cstage_bytes(int nkc, int bn) {
 }
 
 struct Layout {
-    uint32_t x_off, xaug_off, c_off, stage, bar_off, slot_off, merge_off, total;
+    uint32_t x_off, xaug_off, c_off, stage, bar_off, slot_off, delta_off, merge_off, total;
 };
 
 __host__ __device__ inline Layout make_layout(int nkc, int bn, int stages) {
@@ -91,10 +98,12 @@ __host__ __device__ inline Layout make_layout(int nkc, int bn, int stages) {
     L.c_off = L.xaug_off + 2u * XAUG_BYTES;
     L.stage = (cstage_bytes(nkc, bn) + 1023u) & ~1023u;
     L.bar_off = L.c_off + static_cast<uint32_t>(stages) * L.stage;
-    const uint32_t nbar = 11 + 2 * stages;
+    const uint32_t nbar = NUM_BARS_FIXED + 2 * stages;
     L.slot_off = L.bar_off + nbar * 8u;
-    L.merge_off = (L.slot_off + 16u + 15u) & ~15u;
-    L.total = L.merge_off + 2u * BM * 8u;
+    L.delta_off = (L.slot_off + 16u + 15u) & ~15u;
+    L.merge_off = L.delta_off + 2u * BM * 4u;
+    // per point buffer: three column quarters x 128 rows of (value, index)
+    L.total = L.merge_off + 2u * 3u * BM * 8u;
     return L;
 }
 
@@ -151,6 +160,11 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                  : "memory");
 }
+// Remote arrive without release semantics (see mbar_arrive_relaxed).
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
 // 2-SM tensor load: lands in this CTA's shared memory, completes on the leader's barrier.
 __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap *tm,
                                                  uint32_t leader_bar, int c0, int c1, int c2,
@@ -197,35 +211,46 @@ __device__ __forceinline__ void tc_commit_pair_self(uint32_t bar) {
                  : "memory");
 }
 
+// s + lo^2 + hi^2 for the two 16-bit values of `w`, with fp32 accumulation. The square of a
+// 16-bit float is exact in fp32, so this equals converting first and using fmaf; the
+// mixed-precision FMA just needs no conversion instructions.
+template <typename T> __device__ __forceinline__ float sq2_acc(uint32_t w, float s);
+template <> __device__ __forceinline__ float sq2_acc<__half>(uint32_t w, float s) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\t"
+        "fma.rn.f32.f16 %0, l, l, %0;\n\tfma.rn.f32.f16 %0, h, h, %0;\n\t}"
+        : "+f"(s) : "r"(w));
+    return s;
+}
+template <> __device__ __forceinline__ float sq2_acc<__nv_bfloat16>(uint32_t w, float s) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\t"
+        "fma.rn.f32.bf16 %0, l, l, %0;\n\tfma.rn.f32.bf16 %0, h, h, %0;\n\t}"
+        : "+f"(s) : "r"(w));
+    return s;
+}
+
 template <typename T>
-__device__ __forceinline__ float row_sqnorm_swizzled(const uint8_t *row_base) {
-    // A 128-byte row of 64 16-bit values; the swizzle only permutes 16-byte units within the
-    // row, which does not change a sum of squares.
+__device__ __forceinline__ float row_sqnorm_swizzled(const uint8_t *row_base, int row) {
+    // A 128-byte row of 64 16-bit values; the 128-byte swizzle stores logical 16-byte unit u of
+    // row r at position u ^ (r % 8), which a sum of squares does not care about. Reading the
+    // units in that rotated order makes the 32 lanes (32 consecutive rows) of a warp touch all
+    // 32 banks instead of the same 4. Four partial sums keep the FMA chains short.
     const uint4 *rp = reinterpret_cast<const uint4 *>(row_base);
-    float s = 0.f;
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-        const uint4 v = rp[u];
-        const uint32_t wds[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            T lo, hi;
-            const uint16_t l16 = static_cast<uint16_t>(wds[e] & 0xFFFFu);
-            const uint16_t h16 = static_cast<uint16_t>(wds[e] >> 16);
-            memcpy(&lo, &l16, 2);
-            memcpy(&hi, &h16, 2);
-            const float a = Cvt<T>::to_f(lo), c = Cvt<T>::to_f(hi);
-            s = fmaf(a, a, s);
-            s = fmaf(c, c, s);
-        }
+        const uint4 v = rp[u ^ (row & 7)];
+        s[0] = sq2_acc<T>(v.x, s[0]);
+        s[1] = sq2_acc<T>(v.y, s[1]);
+        s[2] = sq2_acc<T>(v.z, s[2]);
+        s[3] = sq2_acc<T>(v.w, s[3]);
     }
-    return s;
+    return (s[0] + s[1]) + (s[2] + s[3]);
 }
 
 template <typename T>
 __device__ __forceinline__ float tile_row_sqnorm(const uint8_t *xbuf, int nkc, int row) {
     float xn = 0.f;
-    for (int kc = 0; kc < nkc; ++kc) xn += row_sqnorm_swizzled<T>(xbuf + kc * XCHUNK + row * 128);
+    for (int kc = 0; kc < nkc; ++kc) xn += row_sqnorm_swizzled<T>(xbuf + kc * XCHUNK + row * 128, row);
     return xn;
 }
 
@@ -241,31 +266,35 @@ __device__ __forceinline__ float min3f(float a, float b, float c) {
     return d;
 }
 
-// Distance bits with the low 5 mantissa bits replaced by the column index inside the chunk.
-__device__ __forceinline__ float key(uint32_t v, uint32_t i) {
-    return __uint_as_float((v & 0xFFFFFFE0u) | i);
-}
-
-// Minimum packed key of a 32-column chunk (four independent chains for ILP).
-__device__ __forceinline__ float chunk_min(const uint32_t (&v)[32]) {
-    float m[4];
+// Minimum packed key over W columns: distance bits with the low log2(W) mantissa bits replaced
+// by the column index (independent chains of eight for ILP).
+template <int W>
+__device__ __forceinline__ float cols_min(const uint32_t (&v)[W]) {
+    constexpr uint32_t MASK = ~static_cast<uint32_t>(W - 1);
+    constexpr int G = W / 8;
+    float m[G];
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
+    for (int g = 0; g < G; ++g) {
         const int o = 8 * g;
-        float t = min3f(key(v[o], o), key(v[o + 1], o + 1), key(v[o + 2], o + 2));
-        t = min3f(t, key(v[o + 3], o + 3), key(v[o + 4], o + 4));
-        t = min3f(t, key(v[o + 5], o + 5), key(v[o + 6], o + 6));
-        m[g] = fminf(t, key(v[o + 7], o + 7));
+        auto key = [&](int i) { return __uint_as_float((v[i] & MASK) | static_cast<uint32_t>(i)); };
+        float t = min3f(key(o), key(o + 1), key(o + 2));
+        t = min3f(t, key(o + 3), key(o + 4));
+        t = min3f(t, key(o + 5), key(o + 6));
+        m[g] = fminf(t, key(o + 7));
     }
-    return fminf(min3f(m[0], m[1], m[2]), m[3]);
+#pragma unroll
+    for (int s = 1; s < G; s *= 2)
+#pragma unroll
+        for (int g = 0; g + s < G; g += 2 * s) m[g] = fminf(m[g], m[g + s]);
+    return m[0];
 }
 
 template <typename T, int BN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     assign_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC,
                      const __grid_constant__ CUtensorMap tmA, const Params p) {
-    constexpr int HALF = BN / 2;        // accumulator columns per epilogue column-half
-    constexpr int NCH = HALF / 32;
+    constexpr int W = BN / 4;           // accumulator columns per epilogue warp
+    constexpr uint32_t IMASK = W - 1;
     constexpr int CROWS = BN / 2;       // centroid rows each CTA stages per tile
     constexpr uint32_t CCHUNK = CROWS * 128u;   // one [bn/2 x 64] centroid chunk
     extern __shared__ uint8_t smem_raw[];
@@ -279,11 +308,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     auto X_FULL = [&](int i) { return bar0 + 8u * i; };
     auto X_EMPTY = [&](int i) { return bar0 + 8u * (2 + i); };
     auto XAUG_FULL = [&](int i) { return bar0 + 8u * (4 + i); };
-    auto ACC_FULL = [&](int i) { return bar0 + 8u * (6 + i); };
-    auto ACC_EMPTY = [&](int i) { return bar0 + 8u * (8 + i); };
-    const uint32_t DRAIN = bar0 + 8u * 10;
-    auto C_FULL = [&](int s) { return bar0 + 8u * (11 + s); };
-    auto C_EMPTY = [&](int s) { return bar0 + 8u * (11 + S + s); };
+    auto DELTA_FULL = [&](int i) { return bar0 + 8u * (6 + i); };
+    auto ACC_FULL = [&](int i) { return bar0 + 8u * (8 + i); };
+    auto ACC_EMPTY = [&](int i) { return bar0 + 8u * (10 + i); };
+    const uint32_t DRAIN = bar0 + 8u * 12;
+    auto C_FULL = [&](int s) { return bar0 + 8u * (NUM_BARS_FIXED + s); };
+    auto C_EMPTY = [&](int s) { return bar0 + 8u * (NUM_BARS_FIXED + S + s); };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -295,9 +325,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         abort_flag = 0;
         for (int i = 0; i < 2; ++i) {
             mbar_init(X_FULL(i), 1);
-            // the leader's commit + own norm warps + own h=0 epilogue warps (distance readers)
-            mbar_init(X_EMPTY(i), 1 + NUM_NORM_WARPS + NUM_EPI_WARPS / 2);
-            mbar_init(XAUG_FULL(i), 2 * NUM_NORM_WARPS);      // (leader) norm warps of both CTAs
+            // own norm warp (done reading the tile) + own column-quarter-0 epilogue warps (the
+            // item's last accumulator seen complete, so every MMA reading the tile is done)
+            mbar_init(X_EMPTY(i), NUM_NORM_WARPS + 4);
+            mbar_init(XAUG_FULL(i), 2 * NUM_NORM_WARPS);      // (leader) norm warp of both CTAs
+            mbar_init(DELTA_FULL(i), NUM_NORM_WARPS);
             mbar_init(ACC_FULL(i), 1);
             mbar_init(ACC_EMPTY(i), 2 * NUM_EPI_WARPS);       // (leader) epilogue warps of both
         }
@@ -387,33 +419,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
     } else if (warp == WARP_MMA) {
         // ------------------------------------------------------------ MMA issuer (leader)
-        if (leader && lane == 0) {
+        if (leader) {
+            const bool issuer = elect_one();   // the same lane issues every MMA and commit
             int stage = 0;
             uint32_t cph = 0;
             int abuf = 0;
             uint32_t aph = 0;
-            bool ok = true;
-            int local = 0;
+            int local = 0, j = 0;
+            int t = cluster_id;
+            bool ready = false;   // the current tile's barriers were already seen complete
             const uint32_t cbase16 = (sbase + L.c_off) >> 4;
             const uint32_t stage16 = L.stage >> 4;
-            const uint32_t cchunk16 = CCHUNK >> 4;
-            for (int t = cluster_id; t < total && ok; t += nclusters, ++local) {
+            constexpr uint32_t cchunk16 = CCHUNK >> 4;
+            const int nk_last = (p.d - (p.nkc - 1) * KC + 15) / 16;   // K steps of the last chunk
+            while (t < total) {
                 const int xb = local & 1;
                 const uint32_t xph = (local >> 1) & 1;
-                // both CTAs' point tiles have landed and their augmentation rows are written
-                if (!mbar_wait(XAUG_FULL(xb), xph, abortp)) { ok = false; break; }
+                if (!ready) {
+                    // both CTAs' point tiles landed and their augmentation rows are written; the
+                    // epilogue has read this accumulator; the centroid tile has landed
+                    if (j == 0 && !mbar_wait_warp(XAUG_FULL(xb), xph, abortp)) break;
+                    if (!mbar_wait_warp(ACC_EMPTY(abuf), aph ^ 1u, abortp)) break;
+                    if (!mbar_wait_warp(C_FULL(stage), cph, abortp)) break;
+                }
+                tc_fence_after();
+                const uint32_t dcol = tmem_base + abuf * ACC_STRIDE;
+                const uint32_t c16 = cbase16 + stage * stage16;
                 const uint32_t x16 = (sbase + L.x_off + xb * p.nkc * XCHUNK) >> 4;
-                const uint32_t xaug16 = (sbase + L.xaug_off + xb * XAUG_BYTES) >> 4;
-                for (int j = 0; j < p.nct; ++j) {
-                    if (!mbar_wait(ACC_EMPTY(abuf), aph ^ 1u, abortp)) { ok = false; break; }
-                    tc_fence_after();   // the epilogue's TMEM reads of this buffer come first
-                    if (!mbar_wait(C_FULL(stage), cph, abortp)) { ok = false; break; }
-                    const uint32_t dcol = tmem_base + abuf * ACC_STRIDE;
-                    const uint32_t c16 = cbase16 + stage * stage16;
+                if (issuer) {
                     uint32_t acc = 0;
                     for (int kc = 0; kc < p.nkc; ++kc) {
-                        const int rem = p.d - kc * KC;
-                        const int nk = rem >= KC ? 4 : (rem + 15) / 16;
+                        const int nk = kc + 1 < p.nkc ? 4 : nk_last;
                         for (int kk = 0; kk < nk; ++kk) {
                             tc_mma_pair(dcol, make_desc(x16 + kc * (XCHUNK >> 4) + kk * 2, DESC_HI_SW128),
                                         make_desc(c16 + kc * cchunk16 + kk * 2, DESC_HI_SW128),
@@ -421,60 +457,90 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                             acc = 1;
                         }
                     }
+                }
+                __syncwarp();
+                // Next tile, and a look at its barriers while this tile's MMAs are queued.
+                int nj = j + 1, nlocal = local, nt = t;
+                if (nj == p.nct) { nj = 0; ++nlocal; nt += nclusters; }
+                const int nstage = stage + 1 == S ? 0 : stage + 1;
+                const uint32_t ncph = stage + 1 == S ? cph ^ 1u : cph;
+                const int nabuf = abuf ^ 1;
+                const uint32_t naph = abuf == 1 ? aph ^ 1u : aph;
+                bool nready = false;
+                if (nt < total) {
+                    nready = mbar_test_wait(ACC_EMPTY(nabuf), naph ^ 1u) &&
+                             mbar_test_wait(C_FULL(nstage), ncph) &&
+                             (nj != 0 || mbar_test_wait(XAUG_FULL(nlocal & 1), (nlocal >> 1) & 1));
+                }
+                ready = __shfl_sync(0xffffffffu, nready ? 1 : 0, 0) != 0;
+                if (issuer) {
+                    const uint32_t xaug16 = (sbase + L.xaug_off + xb * XAUG_BYTES) >> 4;
                     tc_mma_pair(dcol, make_desc(xaug16, DESC_HI_SW32),
                                 make_desc(c16 + p.nkc * cchunk16, DESC_HI_SW32), p.idesc_aug, 1u);
-                    tc_commit_pair_both(C_EMPTY(stage));
                     tc_commit_pair_both(ACC_FULL(abuf));
-                    if (++stage == S) { stage = 0; cph ^= 1u; }
-                    abuf ^= 1;
-                    if (abuf == 0) aph ^= 1u;
                 }
-                if (!ok) break;
-                tc_commit_pair_both(X_EMPTY(xb));
+                __syncwarp();
+                j = nj; local = nlocal; t = nt;
+                stage = nstage; cph = ncph; abuf = nabuf; aph = naph;
             }
             // Every MMA issued above completes before TMEM is released.
-            tc_commit_pair_self(DRAIN);
+            if (issuer) tc_commit_pair_self(DRAIN);
+            __syncwarp();
             mbar_wait(DRAIN, 0, nullptr);
         }
         __syncwarp();
-    } else if (warp >= WARP_NORM0) {
+    } else if (warp < WARP_EPI0) {
         // ------------------------------------------------------------ norms (both CTAs)
-        const int row = (warp - WARP_NORM0) * 32 + lane;
+        const int nw = warp - WARP_NORM0;
+        float *dbuf = reinterpret_cast<float *>(sgen + L.delta_off);
+        const uint32_t xaug_full_leader0 = map_to_rank(XAUG_FULL(0), 0);
+        const uint32_t xaug_full_leader1 = map_to_rank(XAUG_FULL(1), 0);
         int local = 0;
         for (int t = cluster_id; t < total; t += nclusters, ++local) {
             const int xb = local & 1;
             const uint32_t xph = (local >> 1) & 1;
-            if (!mbar_wait(X_FULL(xb), xph, abortp)) break;
-            const float half_xn =
-                0.5f * tile_row_sqnorm<T>(sgen + L.x_off + xb * p.nkc * XCHUNK, p.nkc, row);
-            const float x1 = __bfloat162float(__float2bfloat16_rn(half_xn));
-            const float x2 = __bfloat162float(__float2bfloat16_rn(half_xn - x1));
-            // Row of the point-side augmentation in the 32-byte-swizzled layout: the two 16-byte
-            // halves of rows 4..7 of every 8-row group trade places.
-            const uint4 data = make_uint4(pack_bf16x2(x1, x2), pack_bf16x2(1.f, 1.f),
-                                          pack_bf16x2(1.f, 0.f), 0u);
-            const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-            uint8_t *rp = sgen + L.xaug_off + xb * XAUG_BYTES + row * 32;
-            const int sw = (row >> 2) & 1;
-            *reinterpret_cast<uint4 *>(rp + 16 * sw) = data;
-            *reinterpret_cast<uint4 *>(rp + 16 * (1 - sw)) = zero;
+            if (!mbar_wait_warp(X_FULL(xb), xph, abortp)) break;
+#pragma unroll 1
+            for (int rr = 0; rr < BM / (32 * NUM_NORM_WARPS); ++rr) {
+                const int row = nw * 32 + lane + rr * 32 * NUM_NORM_WARPS;
+                const float half_xn =
+                    0.5f * tile_row_sqnorm<T>(sgen + L.x_off + xb * p.nkc * XCHUNK, p.nkc, row);
+                const float x1 = __bfloat162float(__float2bfloat16_rn(half_xn));
+                const float x2 = __bfloat162float(__float2bfloat16_rn(half_xn - x1));
+                dbuf[xb * BM + row] = (half_xn - x1) - x2;
+                // Row of the point-side augmentation in the 32-byte-swizzled layout: the two
+                // 16-byte halves of rows 4..7 of every 8-row group trade places.
+                const uint4 data = make_uint4(pack_bf16x2(x1, x2), pack_bf16x2(1.f, 1.f),
+                                              pack_bf16x2(1.f, 0.f), 0u);
+                const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+                uint8_t *rp = sgen + L.xaug_off + xb * XAUG_BYTES + row * 32;
+                const int sw = (row >> 2) & 1;
+                *reinterpret_cast<uint4 *>(rp + 16 * sw) = data;
+                *reinterpret_cast<uint4 *>(rp + 16 * (1 - sw)) = zero;
+            }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive_cluster(map_to_rank(XAUG_FULL(xb), 0));
+                mbar_arrive_cluster(xb ? xaug_full_leader1 : xaug_full_leader0);
+                mbar_arrive(DELTA_FULL(xb));
                 mbar_arrive(X_EMPTY(xb));
             }
         }
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int ew = warp - WARP_EPI0;
-        const int q = warp & 3;
-        const int h = ew >> 2;
+        const int q = warp & 3;          // TMEM lane quarter this warp may read
+        const int cq = ew >> 2;          // column quarter of the accumulator
         const int row = q * 32 + lane;
+        const float *dbuf = reinterpret_cast<const float *>(sgen + L.delta_off);
         float *mval = reinterpret_cast<float *>(sgen + L.merge_off);
-        int *midx = reinterpret_cast<int *>(sgen + L.merge_off + 2u * BM * 4u);
+        int *midx = reinterpret_cast<int *>(sgen + L.merge_off + 2u * 3u * BM * 4u);
+        const uint32_t acc_empty_leader0 = map_to_rank(ACC_EMPTY(0), 0);
+        const uint32_t acc_empty_leader1 = map_to_rank(ACC_EMPTY(1), 0);
+        const uint32_t tlane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + cq * W;
         int abuf = 0;
         uint32_t aph = 0;
+        int stage = 0;
         int local = 0;
         for (int t = cluster_id; t < total; t += nclusters, ++local) {
             const int b = t / p.mtiles;
@@ -484,69 +550,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             bool ok = true;
             float best_v = INFINITY;
             int best_i = 0;
-            for (int j = 0; j < p.nct && ok; ++j) {
-                if (!mbar_wait(ACC_FULL(abuf), aph, abortp)) { ok = false; break; }
+            for (int j = 0; j < p.nct; ++j) {
+                if (!mbar_wait_warp(ACC_FULL(abuf), aph, abortp)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t tcol = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                      abuf * ACC_STRIDE + h * HALF;
-                const int kbase = j * BN + h * HALF;
-                uint32_t va[32], vb[32];
-                tmem_ld_32x32b_x32(tcol, va);
-                tmem_wait_ld(va);
-#pragma unroll
-                for (int c = 0; c < NCH; ++c) {
-                    uint32_t(&cur)[32] = (c & 1) ? vb : va;
-                    uint32_t(&nxt)[32] = (c & 1) ? va : vb;
-                    if (c + 1 < NCH) {
-                        tmem_ld_32x32b_x32(tcol + (c + 1) * 32, nxt);
-                    } else {
-                        // every column of this accumulator is in registers: hand it back
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive_cluster(map_to_rank(ACC_EMPTY(abuf), 0));
-                    }
-                    const float m = chunk_min(cur);
-                    const uint32_t mb = __float_as_uint(m);
-                    const float mv = __uint_as_float(mb & 0xFFFFFFE0u);
-                    if (mv < best_v) {
-                        best_v = mv;
-                        best_i = kbase + c * 32 + static_cast<int>(mb & 31u);
-                    }
-                    if (c + 1 < NCH) tmem_wait_ld(nxt);
+                // The tile's MMAs are complete: its centroid stage may be refilled.
+                if (ew == 0 && lane == 0) mbar_arrive_relaxed(C_EMPTY(stage));
+                __syncwarp();
+                uint32_t v[W];
+                if constexpr (W == 64) tmem_ld_32x32b_x64(tlane + abuf * ACC_STRIDE, v);
+                else if constexpr (W == 32) tmem_ld_32x32b_x32(tlane + abuf * ACC_STRIDE, v);
+                else tmem_ld_32x32b_x16(tlane + abuf * ACC_STRIDE, v);
+                tmem_wait_ld(v);
+                // Every column this warp needs is in registers: hand the accumulator back. The
+                // arrive is relaxed, so it never waits for this warp's output stores.
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster_relaxed(abuf ? acc_empty_leader1 : acc_empty_leader0);
+                const float m = cols_min<W>(v);
+                const uint32_t mb = __float_as_uint(m);
+                const float mv = __uint_as_float(mb & ~IMASK);
+                if (mv < best_v) {
+                    best_v = mv;
+                    best_i = j * BN + cq * W + static_cast<int>(mb & IMASK);
                 }
                 abuf ^= 1;
                 if (abuf == 0) aph ^= 1u;
+                if (++stage == S) stage = 0;
             }
-            // The reported distance adds back delta, the rounding of this row's two-piece
-            // ||x||^2/2 split, recomputed from the point tile (still resident: X_EMPTY waits for
-            // these warps too).
+            // Column quarter 0 merges the four quarters of each row and writes the result; the
+            // reported distance adds back delta, the rounding of this row's two-piece ||x||^2/2.
+            const int slot = local & 1;
+            if (cq != 0) {
+                mval[(slot * 3 + cq - 1) * BM + row] = best_v;
+                midx[(slot * 3 + cq - 1) * BM + row] = best_i;
+            }
             float delta = 0.f;
-            if (h == 0) {
-                if (p.need_dist && ok && mbar_wait(X_FULL(xb), xph, abortp)) {
-                    const float half_xn =
-                        0.5f * tile_row_sqnorm<T>(sgen + L.x_off + xb * p.nkc * XCHUNK, p.nkc, row);
-                    const float x1 = __bfloat162float(__float2bfloat16_rn(half_xn));
-                    const float x2 = __bfloat162float(__float2bfloat16_rn(half_xn - x1));
-                    delta = (half_xn - x1) - x2;
-                }
+            if (cq == 0) {
+                if (p.need_dist && ok && mbar_wait_warp(DELTA_FULL(xb), xph, abortp))
+                    delta = dbuf[xb * BM + row];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(X_EMPTY(xb));
             }
-            // Merge the two column halves of each row (both warps of a pair always reach this
-            // barrier once per work item, then leave together if anything gave up).
-            const int mb2 = (local & 1) * BM;
-            if (h == 1) {
-                mval[mb2 + row] = best_v;
-                midx[mb2 + row] = best_i;
-            }
-            named_barrier_sync(1 + q, 64);
-            if (*abortp) break;
-            if (h == 0) {
-                const float ob = mval[mb2 + row];
-                const int oi = midx[mb2 + row];
-                if (ob < best_v || (ob == best_v && oi < best_i)) {
-                    best_v = ob;
-                    best_i = oi;
+            // All four warps of a lane quarter reach this barrier once per work item, then
+            // leave together if any of them saw a role give up.
+            if (named_barrier_or(1 + q, 128, !ok || *abortp != 0)) break;
+            if (cq == 0) {
+#pragma unroll
+                for (int o = 0; o < 3; ++o) {
+                    const float ob = mval[(slot * 3 + o) * BM + row];
+                    const int oi = midx[(slot * 3 + o) * BM + row];
+                    if (ob < best_v) {   // quarters come in column order: ties keep the lower
+                        best_v = ob;
+                        best_i = oi;
+                    }
                 }
                 const int i = m0 + row;
                 double contrib = 0.0;

@@ -18,6 +18,7 @@ __device__ unsigned int g_km_dev_error;
 
 constexpr unsigned int kDevErrTimeout = 1u;
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s
+constexpr uint32_t kSuspendHintNs = 20000u;                  // per blocking probe
 
 // ------------------------------------------------------------------ dtype traits
 
@@ -63,6 +64,19 @@ template <typename V> __device__ __forceinline__ V warp_sum(V v) {
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
+// Named barrier that also returns, to every participant, whether any participant passed true.
+__device__ __forceinline__ bool named_barrier_or(int id, int nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %3, 0;\n\t"
+        "bar.red.or.pred q, %1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(id), "r"(nthreads), "r"(pred ? 1u : 0u)
+        : "memory");
+    return r != 0;
+}
 
 // ------------------------------------------------------------------ mbarrier
 
@@ -72,14 +86,16 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 __device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
+// Blocking probe: the thread is suspended until the phase completes or about `hint_ns` pass,
+// so a waiting warp takes almost no issue slots from the warps that share its scheduler.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
@@ -96,7 +112,8 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 // Bounded wait for the phase with the given parity to complete. `abort_flag` (shared) lets a
-// waiter give up early once another role has given up. Returns false on timeout or abort.
+// waiter give up early once another role has given up (may be null). Returns false on timeout
+// or abort.
 // The first probe does not block, so a wait on a phase that has already completed is cheap.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
     if (mbar_test_wait(bar, parity)) return true;
@@ -106,10 +123,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 #pragma unroll 1
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
+        if (abort_flag && *abort_flag) return false;
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
             record_dev_error(kDevErrTimeout);
-            *abort_flag = 1;
+            if (abort_flag) *abort_flag = 1;
             return false;
         }
     }
@@ -131,6 +148,11 @@ __device__ __forceinline__ bool elect_one() {
 }
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// Arrive without release semantics: for hand-backs that publish no memory writes (a buffer
+// whose reads have completed), so the arrive never waits for this thread's earlier stores.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint32_t bar) {
+    asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
@@ -221,6 +243,48 @@ __device__ __forceinline__ void tmem_wait_ld(uint32_t (&v)[32]) {
                    "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]), "+r"(v[22]), "+r"(v[23]),
                    "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]), "+r"(v[29]),
                    "+r"(v[30]), "+r"(v[31])
+                 :
+                 : "memory");
+}
+
+// 32 lanes x 16 consecutive fp32 columns.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+          "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&v)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                   "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                   "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15])
+                 :
+                 : "memory");
+}
+// 32 lanes x 64 consecutive fp32 columns as two 32-column loads.
+__device__ __forceinline__ void tmem_ld_32x32b_x64(uint32_t taddr, uint32_t (&v)[64]) {
+    uint32_t(&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
+    uint32_t(&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
+    tmem_ld_32x32b_x32(taddr, lo);
+    tmem_ld_32x32b_x32(taddr + 32, hi);
+}
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&v)[64]) {
+    uint32_t(&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
+    uint32_t(&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
+    tmem_wait_ld(lo);
+    // the single wait above covers both loads; this one only pins the upper registers
+    asm volatile("" : "+r"(hi[0]), "+r"(hi[1]), "+r"(hi[2]), "+r"(hi[3]), "+r"(hi[4]), "+r"(hi[5]),
+                      "+r"(hi[6]), "+r"(hi[7]), "+r"(hi[8]), "+r"(hi[9]), "+r"(hi[10]),
+                      "+r"(hi[11]), "+r"(hi[12]), "+r"(hi[13]), "+r"(hi[14]), "+r"(hi[15]),
+                      "+r"(hi[16]), "+r"(hi[17]), "+r"(hi[18]), "+r"(hi[19]), "+r"(hi[20]),
+                      "+r"(hi[21]), "+r"(hi[22]), "+r"(hi[23]), "+r"(hi[24]), "+r"(hi[25]),
+                      "+r"(hi[26]), "+r"(hi[27]), "+r"(hi[28]), "+r"(hi[29]), "+r"(hi[30]),
+                      "+r"(hi[31])
                  :
                  : "memory");
 }
