@@ -135,9 +135,9 @@ struct Params {
 constexpr uint32_t DESC_HI_SW128 = (1024u >> 4) | (1u << 14) | (2u << 29);
 constexpr uint32_t DESC_HI_SW32 = (256u >> 4) | (1u << 14) | (6u << 29);
 constexpr uint32_t DESC_LO_LBO = 1u << 16;
-__device__ __forceinline__ uint64_t make_desc(uint32_t addr16, uint32_t hi) {
-    return (static_cast<uint64_t>(hi) << 32) | (DESC_LO_LBO | (addr16 & 0x3FFFu));
-}
+// Low descriptor word of a shared-memory address (16-byte units; shared memory is below 256 KB,
+// so the 14-bit field never carries into the leading byte offset when offsets are added).
+__device__ __forceinline__ uint32_t desc_lo(uint32_t saddr) { return DESC_LO_LBO | (saddr >> 4); }
 
 // ------------------------------------------------------------------ pair / cluster helpers
 
@@ -187,13 +187,17 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                  : "memory");
 }
-__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                            uint32_t idesc, uint32_t accumulate) {
+// Descriptors passed as (low, high) 32-bit words: only the low word (the start address) changes
+// from one K step to the next.
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
+                                            uint32_t b_lo, uint32_t b_hi, uint32_t idesc,
+                                            uint32_t accumulate) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+        "mov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 // Arrive once on the barrier at this offset in both CTAs of the pair when all MMAs issued so far
@@ -289,7 +293,9 @@ __device__ __forceinline__ float cols_min(const uint32_t (&v)[W]) {
     return m[0];
 }
 
-template <typename T, int BN>
+// NKC = ceil(d / 64): the number of 64-wide chunks of the reduction, fixed per instantiation so
+// the issue loop unrolls into MMAs whose descriptors differ by constants.
+template <typename T, int BN, int NKC>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     assign_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC,
                      const __grid_constant__ CUtensorMap tmA, const Params p) {
@@ -302,7 +308,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
     uint8_t *sgen = smem_raw + (sbase - raw);
-    const Layout L = make_layout(p.nkc, BN, p.stages);
+    const Layout L = make_layout(NKC, BN, p.stages);
     const int S = p.stages;
     const uint32_t bar0 = sbase + L.bar_off;
     auto X_FULL = [&](int i) { return bar0 + 8u * i; };
@@ -356,7 +362,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const int total = p.B * p.mtiles;
     const int cluster_id = blockIdx.x >> 1;
     const int nclusters = gridDim.x >> 1;
-    const uint32_t stage_tx = 2u * cstage_bytes(p.nkc, BN);   // both CTAs' halves of a tile
+    const uint32_t stage_tx = 2u * cstage_bytes(NKC, BN);   // both CTAs' halves of a tile
 
     if (warp == WARP_CPROD) {
         // ------------------------------------------------------------ centroid producer
@@ -374,9 +380,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     if (leader) mbar_arrive_expect_tx(C_FULL(stage), stage_tx);
                     const uint32_t sdst = sbase + L.c_off + stage * L.stage;
                     const uint32_t lbar = map_to_rank(C_FULL(stage), 0);
-                    for (int kc = 0; kc < p.nkc; ++kc)
+                    for (int kc = 0; kc < NKC; ++kc)
                         tma_load_3d_pair(sdst + kc * CCHUNK, &tmC, lbar, kc * KC, crow, b, pol_c);
-                    tma_load_3d_pair(sdst + p.nkc * CCHUNK, &tmA, lbar, 0, crow, b, pol_c);
+                    tma_load_3d_pair(sdst + NKC * CCHUNK, &tmA, lbar, 0, crow, b, pol_c);
                     ++n_c;
                     if (++stage == S) { stage = 0; cph ^= 1u; }
                 }
@@ -403,9 +409,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 const int xb = local & 1;
                 const uint32_t xph = (local >> 1) & 1;
                 if (!mbar_wait(X_EMPTY(xb), xph ^ 1u, abortp)) { ok = false; break; }
-                mbar_arrive_expect_tx(X_FULL(xb), p.nkc * XCHUNK);
-                for (int kc = 0; kc < p.nkc; ++kc)
-                    tma_load_3d(sbase + L.x_off + (xb * p.nkc + kc) * XCHUNK, &tmX, X_FULL(xb),
+                mbar_arrive_expect_tx(X_FULL(xb), NKC * XCHUNK);
+                for (int kc = 0; kc < NKC; ++kc)
+                    tma_load_3d(sbase + L.x_off + (xb * NKC + kc) * XCHUNK, &tmX, X_FULL(xb),
                                 kc * KC, m0, b, pol_x);
                 ++n_x;
             }
@@ -428,10 +434,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             int local = 0, j = 0;
             int t = cluster_id;
             bool ready = false;   // the current tile's barriers were already seen complete
-            const uint32_t cbase16 = (sbase + L.c_off) >> 4;
+            const uint32_t cbase_lo = desc_lo(sbase + L.c_off);
+            const uint32_t xbase_lo = desc_lo(sbase + L.x_off);
+            const uint32_t xaug_lo = desc_lo(sbase + L.xaug_off);
             const uint32_t stage16 = L.stage >> 4;
             constexpr uint32_t cchunk16 = CCHUNK >> 4;
-            const int nk_last = (p.d - (p.nkc - 1) * KC + 15) / 16;   // K steps of the last chunk
+            constexpr uint32_t xchunk16 = XCHUNK >> 4;
+            const int nk_last = (p.d - (NKC - 1) * KC + 15) / 16;   // K steps of the last chunk
             while (t < total) {
                 const int xb = local & 1;
                 const uint32_t xph = (local >> 1) & 1;
@@ -444,19 +453,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 }
                 tc_fence_after();
                 const uint32_t dcol = tmem_base + abuf * ACC_STRIDE;
-                const uint32_t c16 = cbase16 + stage * stage16;
-                const uint32_t x16 = (sbase + L.x_off + xb * p.nkc * XCHUNK) >> 4;
+                const uint32_t b_lo = cbase_lo + stage * stage16;
+                const uint32_t a_lo = xbase_lo + xb * (NKC * xchunk16);
                 if (issuer) {
-                    uint32_t acc = 0;
-                    for (int kc = 0; kc < p.nkc; ++kc) {
-                        const int nk = kc + 1 < p.nkc ? 4 : nk_last;
-                        for (int kk = 0; kk < nk; ++kk) {
-                            tc_mma_pair(dcol, make_desc(x16 + kc * (XCHUNK >> 4) + kk * 2, DESC_HI_SW128),
-                                        make_desc(c16 + kc * cchunk16 + kk * 2, DESC_HI_SW128),
-                                        p.idesc_main, acc);
-                            acc = 1;
-                        }
-                    }
+#pragma unroll
+                    for (int kc = 0; kc < NKC; ++kc)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            if (kc + 1 < NKC || kk < nk_last)
+                                tc_mma_pair(dcol, a_lo + kc * xchunk16 + kk * 2, DESC_HI_SW128,
+                                            b_lo + kc * cchunk16 + kk * 2, DESC_HI_SW128,
+                                            p.idesc_main, (kc | kk) != 0 ? 1u : 0u);
                 }
                 __syncwarp();
                 // Next tile, and a look at its barriers while this tile's MMAs are queued.
@@ -474,9 +481,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 }
                 ready = __shfl_sync(0xffffffffu, nready ? 1 : 0, 0) != 0;
                 if (issuer) {
-                    const uint32_t xaug16 = (sbase + L.xaug_off + xb * XAUG_BYTES) >> 4;
-                    tc_mma_pair(dcol, make_desc(xaug16, DESC_HI_SW32),
-                                make_desc(c16 + p.nkc * cchunk16, DESC_HI_SW32), p.idesc_aug, 1u);
+                    tc_mma_pair(dcol, xaug_lo + xb * (XAUG_BYTES >> 4), DESC_HI_SW32,
+                                b_lo + NKC * cchunk16, DESC_HI_SW32, p.idesc_aug, 1u);
                     tc_commit_pair_both(ACC_FULL(abuf));
                 }
                 __syncwarp();
@@ -486,7 +492,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             // Every MMA issued above completes before TMEM is released.
             if (issuer) tc_commit_pair_self(DRAIN);
             __syncwarp();
-            mbar_wait(DRAIN, 0, nullptr);
+            mbar_wait_warp(DRAIN, 0, nullptr);
         }
         __syncwarp();
     } else if (warp < WARP_EPI0) {
@@ -504,7 +510,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             for (int rr = 0; rr < BM / (32 * NUM_NORM_WARPS); ++rr) {
                 const int row = nw * 32 + lane + rr * 32 * NUM_NORM_WARPS;
                 const float half_xn =
-                    0.5f * tile_row_sqnorm<T>(sgen + L.x_off + xb * p.nkc * XCHUNK, p.nkc, row);
+                    0.5f * tile_row_sqnorm<T>(sgen + L.x_off + xb * NKC * XCHUNK, NKC, row);
                 const float x1 = __bfloat162float(__float2bfloat16_rn(half_xn));
                 const float x2 = __bfloat162float(__float2bfloat16_rn(half_xn - x1));
                 dbuf[xb * BM + row] = (half_xn - x1) - x2;

@@ -131,7 +131,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
         }
     }
 }
-// Warp-wide bounded wait: every lane probes, the warp leaves together (false if any lane gave up).
+// Warp-wide bounded wait (the warp must be converged): every lane probes, the warp leaves
+// together (false if any lane gave up). Measured faster than one lane probing and
+// broadcasting the outcome.
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
     const bool ok = mbar_wait(bar, parity, abort_flag);
     return __all_sync(0xffffffffu, ok);

@@ -219,20 +219,20 @@ km_status run_assign_simt(const void *X, const void *Cx, const float *w, int64_t
     return KM_OK;
 }
 
-template <typename T, int BN>
+template <typename T, int BN, int NKC>
 km_status launch_assign_tc(const CUtensorMap &tmX, const CUtensorMap &tmC, const CUtensorMap &tmA,
                            km::tc::Params &p, int64_t items, cudaStream_t st) {
     using namespace km::tc;
-    p.stages = pick_stages(p.nkc, BN);
+    p.stages = pick_stages(NKC, BN);
     if (p.stages < 2) return KM_ERR_UNSUPPORTED;
-    const Layout L = make_layout(p.nkc, BN, p.stages);
+    const Layout L = make_layout(NKC, BN, p.stages);
     // More than half of the shared memory per block keeps one CTA per SM, so no second CTA
     // ever waits in tcgen05.alloc for the 512 TMEM columns the first one holds.
     const size_t smem = std::max<size_t>(L.total + 1024, SMEM_LIMIT / 2 + 1024);
     // The attribute is an upper bound for every later launch, so it is always set to the
     // kernel's largest request, never to this call's size.
     if (smem > SMEM_ATTR ||
-        cudaFuncSetAttribute(assign_tc_kernel<T, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(assign_tc_kernel<T, BN, NKC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(SMEM_ATTR)) != cudaSuccess)
         return KM_ERR_CUDA;
     // Persistent clusters (SM pairs): as many as can be resident at once (a pair needs two SMs
@@ -253,7 +253,7 @@ km_status launch_assign_tc(const CUtensorMap &tmX, const CUtensorMap &tmC, const
         attr.val.clusterDim.z = 1;
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
-        if (cudaOccupancyMaxActiveClusters(&max_clusters, assign_tc_kernel<T, BN>, &cfg) != cudaSuccess ||
+        if (cudaOccupancyMaxActiveClusters(&max_clusters, assign_tc_kernel<T, BN, NKC>, &cfg) != cudaSuccess ||
             max_clusters <= 0) {
             cudaGetLastError();
             max_clusters = std::max(1, num_sms() / 2);
@@ -262,7 +262,7 @@ km_status launch_assign_tc(const CUtensorMap &tmX, const CUtensorMap &tmC, const
     }
     const int64_t clusters = std::min<int64_t>(items, max_clusters);
     const unsigned grid = static_cast<unsigned>(2 * clusters);
-    assign_tc_kernel<T, BN><<<grid, NUM_THREADS, smem, st>>>(tmX, tmC, tmA, p);
+    assign_tc_kernel<T, BN, NKC><<<grid, NUM_THREADS, smem, st>>>(tmX, tmC, tmA, p);
     return launch_status();
 }
 
@@ -338,11 +338,14 @@ km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float 
     p.inertia = inertia;
     const int64_t items = B * p.mtiles;
     if (items > kMaxIndex) return KM_ERR_UNSUPPORTED;
-    switch (bn) {
-        case 64: return launch_assign_tc<T, 64>(tmX, tmC, tmA, p, items, st);
-        case 128: return launch_assign_tc<T, 128>(tmX, tmC, tmA, p, items, st);
-        default: return launch_assign_tc<T, 256>(tmX, tmC, tmA, p, items, st);
-    }
+    // (bn, chunks of 64 along d); bn = 256 with d > 192 never fits (tc_bn narrows it)
+#define KM_TC_CASE(BN_, NKC_) \
+    if (bn == BN_ && nkc == NKC_) return launch_assign_tc<T, BN_, NKC_>(tmX, tmC, tmA, p, items, st);
+    KM_TC_CASE(64, 1) KM_TC_CASE(64, 2) KM_TC_CASE(64, 3) KM_TC_CASE(64, 4)
+    KM_TC_CASE(128, 1) KM_TC_CASE(128, 2) KM_TC_CASE(128, 3) KM_TC_CASE(128, 4)
+    KM_TC_CASE(256, 1) KM_TC_CASE(256, 2) KM_TC_CASE(256, 3)
+#undef KM_TC_CASE
+    return KM_ERR_UNSUPPORTED;
 }
 
 // Validated-argument assignment; `caug` must hold ws_assign(B, K, d) bytes when the tensor-core
@@ -370,14 +373,29 @@ template <typename T, int VEC, int G>
 km_status run_segreduce_t(const void *X, const float *w, const int32_t *perm,
                           const int32_t *offsets, int64_t B, int64_t N, int64_t K, int64_t d,
                           float *sums, float *wsum, cudaStream_t st) {
-    const int64_t total = B * N;
-    const int64_t target = static_cast<int64_t>(num_sms()) * 48;
-    int64_t range = ceil_div(total, target);
-    range = std::max<int64_t>(256, ceil_div(range, 32) * 32);
-    range = std::min<int64_t>(range, ceil_div(N, 32) * 32);
+    // One wave: as many (warp, range) pairs as warps that can be resident at once, split
+    // evenly over the batch elements (each warp walks one contiguous range of sorted positions).
+    const int64_t ycols = ceil_div(d, static_cast<int64_t>(G) * VEC);
+    static int blocks_per_sm[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int bps = (dev >= 0 && dev < 64) ? blocks_per_sm[dev] : 0;
+    if (bps <= 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, km::upd::segreduce_kernel<T, VEC, G>,
+                                                          km::upd::SEG_THREADS, 0) != cudaSuccess ||
+            bps <= 0) {
+            cudaGetLastError();
+            bps = 1;
+        }
+        if (dev >= 0 && dev < 64) blocks_per_sm[dev] = bps;
+    }
+    const int64_t resident_warps = static_cast<int64_t>(num_sms()) * bps * (km::upd::SEG_THREADS / 32);
+    const int64_t want = std::max<int64_t>(1, resident_warps / ycols);
+    const int64_t rpb0 = std::max<int64_t>(1, want / B);
+    int64_t range = ceil_div(N, rpb0);
+    range = std::max<int64_t>(64, ceil_div(range, 32) * 32);
     const int64_t rpb = ceil_div(N, range);
     const int64_t warps = B * rpb;
-    const int64_t ycols = ceil_div(d, static_cast<int64_t>(G) * VEC);
     dim3 grid(static_cast<unsigned>(ceil_div(warps, km::upd::SEG_THREADS / 32)),
               static_cast<unsigned>(ycols));
     if (ycols > kMaxGridY) return KM_ERR_UNSUPPORTED;
@@ -386,6 +404,45 @@ km_status run_segreduce_t(const void *X, const float *w, const int32_t *perm,
         static_cast<int>(K), static_cast<int>(d), static_cast<int>(range), static_cast<int>(rpb),
         sums, wsum);
     return launch_status();
+}
+
+// The row-per-warp form (d = 32 * V): one wave of (warp, range) pairs, split evenly over the
+// batch elements.
+template <typename T, int V, bool WEIGHTED>
+km_status run_segreduce_rows_w(const void *X, const float *w, const int32_t *perm,
+                             const int32_t *offsets, int64_t B, int64_t N, int64_t K,
+                             float *sums, float *wsum, cudaStream_t st) {
+    using namespace km::upd;
+    static int blocks_per_sm[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int bps = (dev >= 0 && dev < 64) ? blocks_per_sm[dev] : 0;
+    if (bps <= 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, segreduce_rows_kernel<T, V, WEIGHTED>, ROWS_THREADS, 0) !=
+                cudaSuccess ||
+            bps <= 0) {
+            cudaGetLastError();
+            bps = 1;
+        }
+        if (dev >= 0 && dev < 64) blocks_per_sm[dev] = bps;
+    }
+    const int64_t resident_warps = static_cast<int64_t>(num_sms()) * bps * (ROWS_THREADS / 32);
+    const int64_t rpb0 = std::max<int64_t>(1, resident_warps / B);
+    const int64_t range = std::max<int64_t>(64, ceil_div(ceil_div(N, rpb0), 32) * 32);
+    const int64_t rpb = ceil_div(N, range);
+    const int64_t warps = B * rpb;
+    segreduce_rows_kernel<T, V, WEIGHTED><<<static_cast<unsigned>(ceil_div(warps, ROWS_THREADS / 32)), ROWS_THREADS, 0, st>>>(
+        static_cast<const T *>(X), w, perm, offsets, static_cast<int>(B), static_cast<int>(N),
+        static_cast<int>(K), static_cast<int>(range), static_cast<int>(rpb), sums, wsum);
+    return launch_status();
+}
+template <typename T, int V>
+km_status run_segreduce_rows(const void *X, const float *w, const int32_t *perm,
+                             const int32_t *offsets, int64_t B, int64_t N, int64_t K,
+                             float *sums, float *wsum, cudaStream_t st) {
+    // the weight sums are produced exactly when weights are given
+    if (w) return run_segreduce_rows_w<T, V, true>(X, w, perm, offsets, B, N, K, sums, wsum, st);
+    return run_segreduce_rows_w<T, V, false>(X, w, perm, offsets, B, N, K, sums, wsum, st);
 }
 
 template <typename T, int VEC>
@@ -412,6 +469,14 @@ km_status segreduce_dispatch(const void *X, const float *w, const int32_t *perm,
     int64_t lanes = ceil_div(d, vw);
     int G = 1;
     while (G < lanes && G < 32) G <<= 1;
+    // row-per-warp form: lane l owns columns [l * V, l * V + V), V = d / 32, with V * sizeof(T)
+    // of 4, 8 or 16 bytes (aligned loads and, for 16 bytes of fp32, vector atomics)
+    if (d % 32 == 0 && aligned(X, 16) && aligned(sums, 16)) {
+        const int64_t vb = (d / 32) * static_cast<int64_t>(sizeof(T));
+        if (vb == 4) return run_segreduce_rows<T, 4 / sizeof(T)>(X, w, perm, offsets, B, N, K, sums, wsum, st);
+        if (vb == 8) return run_segreduce_rows<T, 8 / sizeof(T)>(X, w, perm, offsets, B, N, K, sums, wsum, st);
+        if (vb == 16) return run_segreduce_rows<T, 16 / sizeof(T)>(X, w, perm, offsets, B, N, K, sums, wsum, st);
+    }
     if (vec) return segreduce_g<T, VV>(G, X, w, perm, offsets, B, N, K, d, sums, wsum, st);
     return segreduce_g<T, 1>(G, X, w, perm, offsets, B, N, K, d, sums, wsum, st);
 }

@@ -12,6 +12,9 @@
 //              registers while the cluster id stays the same, and merges each run into
 //              sums[B,K,d] with vector atomics (red.global.add.v4.f32): one per run per
 //              4-column group, i.e. O((K + N/range) * d) atomics instead of O(N * d).
+//              Two forms: segreduce_rows_kernel for d = 32 * V (one warp load per row, the run
+//              logic warp-uniform, many warps per SM to keep the random row gathers in flight)
+//              and segreduce_kernel for any other d (G lanes per row, column blocks).
 //
 // The order of points inside a segment is not fixed (tiles reserve their slots atomically), so
 // fp32 sums may differ in the last bits from run to run; the set of points per segment, the
@@ -19,6 +22,8 @@
 #pragma once
 
 #include <limits.h>
+
+#include <type_traits>
 
 #include "km_common.cuh"
 
@@ -30,6 +35,7 @@ constexpr int TILE_THREADS = 512;
 constexpr int SMEM_K_MAX = 16384;   // bins kept in shared memory
 constexpr int SCAN_THREADS = 1024;
 constexpr int SEG_THREADS = 256;
+constexpr int SEG_BLOCKS_PER_SM = 2;
 
 __global__ void __launch_bounds__(TILE_THREADS)
     hist_kernel(const int32_t *__restrict__ ids, int N, int K, int32_t *__restrict__ counts,
@@ -154,13 +160,14 @@ template <typename T, int VEC> struct alignas(sizeof(T) * VEC) VecT {
     T v[VEC];
 };
 
+// The reducing kernels never read the sums back, so the vector reduction carries no memory
+// clobber and loads may be scheduled across it.
 template <int VEC> __device__ __forceinline__ void red_add_row(float *dst, const float (&a)[VEC]) {
     if constexpr (VEC % 4 == 0) {
 #pragma unroll
         for (int e = 0; e < VEC; e += 4)
             asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + e), "f"(a[e]),
-                         "f"(a[e + 1]), "f"(a[e + 2]), "f"(a[e + 3])
-                         : "memory");
+                         "f"(a[e + 1]), "f"(a[e + 2]), "f"(a[e + 3]));
     } else {
 #pragma unroll
         for (int e = 0; e < VEC; ++e) atomicAdd(dst + e, a[e]);
@@ -170,14 +177,22 @@ template <int VEC> __device__ __forceinline__ void red_add_row(float *dst, const
 // G lanes cooperate on one row (G a power of two), each lane covering VEC consecutive columns;
 // a warp handles 32 / G rows per step. Column block blockIdx.y covers columns
 // [blockIdx.y * G * VEC, +G * VEC).
+//
+// Per chunk of 32 sorted positions the warp loads the chunk's point indices (prefetched one
+// chunk ahead), issues the row gathers at once (SB rows per lane in flight), and only then
+// looks up the segment (cluster) of each position, so the lookup's reads of the offsets
+// overlap the gathers instead of delaying them.
 template <typename T, int VEC, int G>
-__global__ void __launch_bounds__(SEG_THREADS, 3)
+__global__ void __launch_bounds__(SEG_THREADS, SEG_BLOCKS_PER_SM)
     segreduce_kernel(const T *__restrict__ X, const float *__restrict__ w,
                      const int32_t *__restrict__ perm, const int32_t *__restrict__ offsets, int B,
                      int N, int K, int d, int range, int ranges_per_batch, float *__restrict__ sums,
                      float *__restrict__ wsum) {
     constexpr int NG = 32 / G;           // rows per warp step
-    constexpr int SB = G < 8 ? G : 8;    // rows gathered per lane before they are consumed
+    // rows gathered per lane before they are consumed (bf16 rows take more registers to
+    // convert, so fewer are kept in flight there)
+    constexpr int SBMAX = std::is_same<T, __nv_bfloat16>::value ? 8 : 16;
+    constexpr int SB = G < SBMAX ? G : SBMAX;
     constexpr unsigned FULL = 0xffffffffu;
     const int lane = threadIdx.x & 31;
     const int64_t gw = static_cast<int64_t>(blockIdx.x) * (SEG_THREADS / 32) + (threadIdx.x >> 5);
@@ -216,41 +231,22 @@ __global__ void __launch_bounds__(SEG_THREADS, 3)
         if (wsb && lg == 0 && blockIdx.y == 0) atomicAdd(wsb + k, wacc);
     };
 
+    int next_i = permb[min(p0 + lane, p1 - 1)];
     for (int q = p0; q < p1; q += 32) {
         const int pl = min(q + lane, p1 - 1);
-        const int my_i = permb[pl];
+        const int my_i = next_i;
+        if (q + 32 < p1) next_i = permb[min(q + 32 + lane, p1 - 1)];
         const float my_w = wb ? wb[my_i] : 1.f;
-        // segment of pl = kcur + #{j >= 1 : offb[kcur + j] <= pl}; 32 offsets per probe round
-        int base = kcur, my_k = -1;
-        while (true) {
-            const int idx = base + 1 + lane;
-            const int o = idx <= K ? offb[idx] : INT_MAX;
-            int cnt = 0;
-#pragma unroll
-            for (int st = 16; st > 0; st >>= 1) {
-                const int pr = __shfl_sync(FULL, o, cnt + st - 1);
-                if (pr <= pl) cnt += st;
-            }
-            const int o31 = __shfl_sync(FULL, o, 31);
-            if (cnt == 31 && o31 <= pl) cnt = 32;
-            if (my_k < 0 && cnt < 32) my_k = base + cnt;
-            if (!__any_sync(FULL, my_k < 0)) break;
-            base += 32;
-        }
-        kcur = __shfl_sync(FULL, my_k, 31);
+        int kseg = 0;
 
 #pragma unroll
         for (int s0 = 0; s0 < G; s0 += SB) {
             VecT<T, VEC> xv[SB];
-            int kk[SB];
-            float wv[SB];
             bool rv[SB];
 #pragma unroll
             for (int s = 0; s < SB; ++s) {
                 const int rr = (s0 + s) * NG + g;
                 const int ii = __shfl_sync(FULL, my_i, rr);
-                kk[s] = __shfl_sync(FULL, my_k, rr);
-                wv[s] = __shfl_sync(FULL, my_w, rr);
                 rv[s] = q + rr < p1;
                 if (rv[s] && colok) {
                     xv[s] = *reinterpret_cast<const VecT<T, VEC> *>(Xb + static_cast<int64_t>(ii) * d + col);
@@ -259,19 +255,177 @@ __global__ void __launch_bounds__(SEG_THREADS, 3)
                     for (int e = 0; e < VEC; ++e) xv[s].v[e] = Cvt<T>::from_f(0.f);
                 }
             }
+            if (s0 == 0) {
+                // segment of pl = kcur + #{j >= 1 : offb[kcur + j] <= pl}; 32 offsets per probe
+                // round (runs while the gathers above are in flight)
+                int base = kcur, my_k = -1;
+                while (true) {
+                    const int idx = base + 1 + lane;
+                    const int o = idx <= K ? offb[idx] : INT_MAX;
+                    int cnt = 0;
+#pragma unroll
+                    for (int st = 16; st > 0; st >>= 1) {
+                        const int pr = __shfl_sync(FULL, o, cnt + st - 1);
+                        if (pr <= pl) cnt += st;
+                    }
+                    const int o31 = __shfl_sync(FULL, o, 31);
+                    if (cnt == 31 && o31 <= pl) cnt = 32;
+                    if (my_k < 0 && cnt < 32) my_k = base + cnt;
+                    if (!__any_sync(FULL, my_k < 0)) break;
+                    base += 32;
+                }
+                kcur = __shfl_sync(FULL, my_k, 31);
+                kseg = my_k;
+            }
 #pragma unroll
             for (int s = 0; s < SB; ++s) {
+                const int rr = (s0 + s) * NG + g;
+                const int kk = __shfl_sync(FULL, kseg, rr);
+                const float wv = __shfl_sync(FULL, my_w, rr);
                 if (rv[s]) {
-                    if (kk[s] != acck) {
+                    if (kk != acck) {
                         if (acck >= 0) flush(acck);
-                        acck = kk[s];
+                        acck = kk;
 #pragma unroll
                         for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
                         wacc = 0.f;
                     }
 #pragma unroll
-                    for (int e = 0; e < VEC; ++e) acc[e] = fmaf(wv[s], Cvt<T>::to_f(xv[s].v[e]), acc[e]);
-                    wacc += wv[s];
+                    for (int e = 0; e < VEC; ++e) acc[e] = fmaf(wv, Cvt<T>::to_f(xv[s].v[e]), acc[e]);
+                    wacc += wv;
+                }
+            }
+        }
+    }
+    if (acck >= 0) flush(acck);
+}
+
+// The segmented reduction for d = 32 * V (V * sizeof(T) of 4, 8 or 16 bytes): lane l of a warp
+// owns columns [l * V, l * V + V), so one warp load fetches one whole row (coalesced) and the
+// cluster of a row, the end of a run and the flush are warp-uniform (one vector atomic per lane
+// per run). Each warp walks chunks of 32 sorted positions; the chunk's point indices are
+// fetched one chunk ahead, and its rows are loaded R at a time into registers (R rows of
+// V * sizeof(T) bytes per lane = 4 KB per warp) before any of them is summed. With few
+// registers per thread many warps fit on an SM, which is what keeps enough bytes in flight
+// for random row gathers to run at HBM speed.
+constexpr int ROWS_THREADS = 256;
+constexpr int ROWS_BLOCKS_PER_SM = 4;
+
+template <typename T, int V, bool WEIGHTED>
+__global__ void __launch_bounds__(ROWS_THREADS, ROWS_BLOCKS_PER_SM)
+    segreduce_rows_kernel(const T *__restrict__ X, const float *__restrict__ w,
+                          const int32_t *__restrict__ perm, const int32_t *__restrict__ offsets,
+                          int B, int N, int K, int range, int ranges_per_batch,
+                          float *__restrict__ sums, float *__restrict__ wsum) {
+    constexpr unsigned FULL = 0xffffffffu;
+    constexpr int d = 32 * V;
+    constexpr int R = 128 / static_cast<int>(V * sizeof(T));   // rows in flight per lane
+    const int lane = threadIdx.x & 31;
+    const int64_t gw = static_cast<int64_t>(blockIdx.x) * (ROWS_THREADS / 32) + (threadIdx.x >> 5);
+    if (gw >= static_cast<int64_t>(B) * ranges_per_batch) return;
+    const int b = static_cast<int>(gw / ranges_per_batch);
+    const int32_t *offb = offsets + static_cast<int64_t>(b) * (K + 1);
+    const int p0 = static_cast<int>(gw % ranges_per_batch) * range;
+    const int p1 = min(offb[K], p0 + range);
+    if (p0 >= p1) return;
+    const int nchunks = (p1 - p0 + 31) / 32;
+    const int col = lane * V;
+    const int32_t *permb = perm + static_cast<int64_t>(b) * N;
+    const T *Xb = X + static_cast<int64_t>(b) * N * d + col;
+    const float *wb = WEIGHTED ? w + static_cast<int64_t>(b) * N : nullptr;
+    float *sb = sums + static_cast<int64_t>(b) * K * d + col;
+    float *wsb = wsum ? wsum + static_cast<int64_t>(b) * K : nullptr;   // wanted with or without weights
+
+    // segment holding p0: the largest k with offb[k] <= p0 (offb[0] = 0, offb[K] = N > p0)
+    int lo = 0, hi = K - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (offb[mid] <= p0) lo = mid; else hi = mid - 1;
+    }
+    int kcur = lo;
+
+    float acc[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) acc[e] = 0.f;
+    float wacc = 0.f;
+    int acck = -1;
+    auto flush = [&](int k) {
+        red_add_row<V>(sb + static_cast<int64_t>(k) * d, acc);
+        if (wsb && lane == 0) atomicAdd(wsb + k, wacc);
+    };
+
+    auto load_idx = [&](int c) {
+        const int pos = p0 + 32 * c + lane;
+        return (c < nchunks && pos < p1) ? permb[pos] : -1;
+    };
+    int idx_next = load_idx(0);
+    for (int c = 0; c < nchunks; ++c) {
+        const int my_i = idx_next;
+        idx_next = load_idx(c + 1);
+        const int q = p0 + 32 * c;
+        const int nrows = min(32, p1 - q);
+        unsigned starts = 0;
+        int my_k = 0;
+        float my_w = 1.f;
+#pragma unroll 1
+        for (int h = 0; h < 32; h += R) {
+            if (h < nrows) {   // warp-uniform
+                VecT<T, V> xv[R];
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const int ri = __shfl_sync(FULL, my_i, h + r);
+                    if (h + r < nrows) xv[r] = *reinterpret_cast<const VecT<T, V> *>(Xb + static_cast<int64_t>(ri) * d);
+                }
+                if (h == 0) {
+                    // clusters of the chunk's positions, while the first rows are in flight:
+                    // segment of pl = kcur + #{j >= 1 : offb[kcur + j] <= pl}
+                    const int pl = min(q + lane, p1 - 1);
+                    int base = kcur;
+                    my_k = -1;
+                    while (true) {
+                        const int idx = base + 1 + lane;
+                        const int o = idx <= K ? offb[idx] : INT_MAX;
+                        int cnt = 0;
+#pragma unroll
+                        for (int stp = 16; stp > 0; stp >>= 1) {
+                            const int pr = __shfl_sync(FULL, o, cnt + stp - 1);
+                            if (pr <= pl) cnt += stp;
+                        }
+                        const int o31 = __shfl_sync(FULL, o, 31);
+                        if (cnt == 31 && o31 <= pl) cnt = 32;
+                        if (my_k < 0 && cnt < 32) my_k = base + cnt;
+                        if (!__any_sync(FULL, my_k < 0)) break;
+                        base += 32;
+                    }
+                    kcur = __shfl_sync(FULL, my_k, 31);
+                    if (WEIGHTED) my_w = my_i >= 0 ? wb[my_i] : 0.f;
+                    // rows that start a new run (their cluster differs from the previous row's)
+                    int prev_k = __shfl_up_sync(FULL, my_k, 1);
+                    if (lane == 0) prev_k = acck;
+                    starts = __ballot_sync(FULL, lane < nrows && my_k != prev_k);
+                }
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const int rr = h + r;
+                    if (rr < nrows) {   // warp-uniform
+                        if ((starts >> rr) & 1u) {   // warp-uniform, about once per run
+                            if (acck >= 0) flush(acck);
+                            acck = __shfl_sync(FULL, my_k, rr);
+#pragma unroll
+                            for (int e = 0; e < V; ++e) acc[e] = 0.f;
+                            wacc = 0.f;
+                        }
+                        if constexpr (WEIGHTED) {
+                            const float wv = __shfl_sync(FULL, my_w, rr);
+#pragma unroll
+                            for (int e = 0; e < V; ++e) acc[e] = fmaf(wv, Cvt<T>::to_f(xv[r].v[e]), acc[e]);
+                            wacc += wv;
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < V; ++e) acc[e] += Cvt<T>::to_f(xv[r].v[e]);
+                            wacc += 1.f;
+                        }
+                    }
                 }
             }
         }
