@@ -39,7 +39,7 @@ ASSIGN_FLOP = 2.0 * B * N * K * D                       # <x,c> contraction per 
 # algorithmic bytes of the update: X gathered once + ids read twice + perm written and read
 UPDATE_BYTES = B * N * D * 2 + 4 * B * N * 4 + B * K * D * 4 * 2
 ASSIGN_BYTES = B * N * D * 2 + B * K * D * 2 + B * N * 4
-LAUNCHES_PER_STEP = 8   # cnpad, assign_tc, hist, scan, scatter, segreduce, finalize, prep
+LAUNCHES_PER_STEP = 8   # caug, assign_tc, hist, scan, scatter, segreduce, finalize, prep
 
 
 def _peaks():
@@ -234,7 +234,7 @@ def run_gpu(args):
             "assign_pt_k_per_s": ws * B * N * K / (assign_ms * 1e-3),
             "assign_ms": assign_ms,
             "update_ms": update_ms,
-            "roofline": {"bound": "tensor", "kernel": "assign_tc_kernel (+ norm padding)",
+            "roofline": {"bound": "tensor", "kernel": "assign_tc_kernel (+ caug_kernel, the centroid side of the norm step)",
                          "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": achieved_tf / peak_tf, "traffic": traffic,
                          "peak_source": f"{peak_kind} bf16 dense (fp16 nominal ratio 1.0)"},

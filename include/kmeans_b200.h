@@ -96,7 +96,10 @@ km_status km_prep(const float *C, km_dtype dtype, int64_t B, int64_t K, int64_t 
  * evaluates sum_j (x_j - c_j)^2 directly. On the tensor-core path mind is formed as
  * ||x||^2 + (||c||^2 - 2<x,c>) in fp32, so its absolute error is a small multiple of
  * 2^-24 (||x||^2 + ||c||^2); for points almost on their centroid that can exceed 1e-4 of the
- * distance itself (the assignment is unaffected except at near-ties).
+ * distance itself (the assignment is unaffected except at near-ties). The tensor-core path also
+ * compares distances as packed (value, index) keys whose lowest 4-6 mantissa bits hold the
+ * column: distances closer than 2^-17 relative are resolved by index, and the reported mind is
+ * truncated by less than 2^-17 relative.
  */
 km_status km_assign(const void *X, km_dtype dtype, const void *Cx, const float *cn,
                     const float *w, int64_t B, int64_t N, int64_t K, int64_t d, int32_t *ids,
