@@ -32,24 +32,30 @@
 // Keeping the tensor pipe fed. The MMA queue holds only a couple of instructions, so whatever
 // the issuing warp does between the last MMA of one tile and the first of the next is a bubble.
 // That gap is kept to one commit: a ring stage holds a whole centroid tile behind one barrier,
-// the stage and the point buffer are handed back by the epilogue (which has seen the tile's
-// completion) rather than by further commits, and the next tile's barriers are probed while the
-// current tile's MMAs are still queued. The MMA warp runs converged and issues from one elected
-// lane, so its addresses and descriptors stay warp-uniform.
+// and the stage and the point buffer are handed back by the epilogue (which has seen the tile's
+// completion) rather than by further commits. An MMA warp runs converged and issues from one
+// elected lane, so its addresses and descriptors stay warp-uniform.
 //
 // Keeping the epilogue off the critical path. TMEM loads have a long latency, so each epilogue
 // warp issues all of its columns of a tile at once (one wait per tile) and sixteen warps share
 // the accumulator: four TMEM lane quarters x four column quarters. The accumulator is released
 // as soon as the registers hold it; the min/argmin math runs while the next tile is computed.
 //
+// Issuing MMAs costs the SM sub-partition that hosts the issuing warp a large share of its
+// issue slots (measured: the epilogue warps beside it finish their tiles last), so two warps
+// on different sub-partitions take turns: tile j is issued by the warp that owns accumulator
+// j % 2.
+//
 // Roles per CTA (persistent clusters, 20 warps: five per SM sub-partition, which leaves 96
 // registers per thread):
 //   warp 0      centroid producer: own half of each centroid tile [bn/2 x d] and its augmentation
 //               rows [bn/2 x 16] into one stage of a ring (L2 evict-last: every CTA re-reads them).
-//   warp 1      TMEM allocation (512 columns, both CTAs); in the leader also the MMA issuer.
-//   warp 2      point producer: own point tile [128 x d], double-buffered (L2 evict-first).
-//   warp 3      norms: ||x||^2 of the point tile as soon as it lands, the point-side augmentation
-//               rows and delta, so the MMA never waits for the epilogue between work items.
+//   warp 1      TMEM allocation (512 columns, both CTAs); in the leader the MMA issuer for even
+//               tiles (accumulator 0).
+//   warp 2      point producer: own point tile [128 x d], double-buffered (L2 evict-first); then
+//               ||x||^2 of the tile as soon as it lands, the point-side augmentation rows and
+//               delta, so the MMA never waits for the epilogue between work items.
+//   warp 3      in the leader the MMA issuer for odd tiles (accumulator 1).
 //   warps 4-19  epilogue: TMEM lane quarter = warp % 4, column quarter = (warp - 4) / 4; one point
 //               row per thread.
 //
@@ -68,12 +74,11 @@ constexpr int KC = 64;                      // 16-bit elements per 128-byte swiz
 constexpr uint32_t XCHUNK = BM * 128;       // bytes of one [128 x 64] point chunk
 constexpr uint32_t XAUG_BYTES = BM * 32;    // [128 x 16] bf16 point-side augmentation
 constexpr int NUM_EPI_WARPS = 16;
-constexpr int NUM_NORM_WARPS = 1;
 constexpr int WARP_CPROD = 0;
-constexpr int WARP_MMA = 1;
-constexpr int WARP_XPROD = 2;
-constexpr int WARP_NORM0 = 3;
-constexpr int WARP_EPI0 = WARP_NORM0 + NUM_NORM_WARPS;
+constexpr int WARP_MMA = 1;       // even tiles (accumulator 0); allocates TMEM
+constexpr int WARP_XPROD = 2;     // point tiles and their norms
+constexpr int WARP_MMA_ODD = 3;   // odd tiles (accumulator 1)
+constexpr int WARP_EPI0 = 4;
 constexpr int NUM_THREADS = 32 * (WARP_EPI0 + NUM_EPI_WARPS);
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_STRIDE = 256;        // TMEM columns between the two accumulators
@@ -120,6 +125,7 @@ struct Params {
     int nct;      // centroid tiles: Kp / bn
     int mtiles;   // 256-point pair tiles per batch: ceil(N / 256)
     int stages;   // centroid ring depth
+    int resident; // 1 when stages == nct: centroid tiles stay in shared memory per batch element
     int need_dist;  // 1 when the distance / inertia is requested
     uint32_t idesc_main, idesc_aug;
     const float *w;
@@ -331,15 +337,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         abort_flag = 0;
         for (int i = 0; i < 2; ++i) {
             mbar_init(X_FULL(i), 1);
-            // own norm warp (done reading the tile) + own column-quarter-0 epilogue warps (the
+            // own point warp (done reading the tile) + own column-quarter-0 epilogue warps (the
             // item's last accumulator seen complete, so every MMA reading the tile is done)
-            mbar_init(X_EMPTY(i), NUM_NORM_WARPS + 4);
-            mbar_init(XAUG_FULL(i), 2 * NUM_NORM_WARPS);      // (leader) norm warp of both CTAs
-            mbar_init(DELTA_FULL(i), NUM_NORM_WARPS);
+            mbar_init(X_EMPTY(i), 1 + 4);
+            mbar_init(XAUG_FULL(i), 2);      // (leader) point warp of both CTAs
+            mbar_init(DELTA_FULL(i), 1);
             mbar_init(ACC_FULL(i), 1);
             mbar_init(ACC_EMPTY(i), 2 * NUM_EPI_WARPS);       // (leader) epilogue warps of both
         }
-        mbar_init(DRAIN, 1);
+        mbar_init(DRAIN, 2);   // one commit per MMA warp
         for (int s = 0; s < S; ++s) {
             mbar_init(C_FULL(s), 1);
             mbar_init(C_EMPTY(s), 1);
@@ -360,8 +366,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(sgen + L.slot_off);
     const int total = p.B * p.mtiles;
+    // Each cluster takes a contiguous range of work items, so it changes batch element (and,
+    // with resident centroids, reloads them) as rarely as possible.
     const int cluster_id = blockIdx.x >> 1;
     const int nclusters = gridDim.x >> 1;
+    const int per_cluster = (total + nclusters - 1) / nclusters;
+    const int t_begin = min(total, cluster_id * per_cluster);
+    const int t_end = min(total, t_begin + per_cluster);
     const uint32_t stage_tx = 2u * cstage_bytes(NKC, BN);   // both CTAs' halves of a tile
 
     if (warp == WARP_CPROD) {
@@ -372,11 +383,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             uint32_t cph = 0;
             long long n_c = 0;
             bool ok = true;
-            for (int t = cluster_id; t < total && ok; t += nclusters) {
+            int cur_b = -1;   // batch element whose centroid tiles the ring holds (resident mode)
+            for (int t = t_begin; t < t_end && ok; ++t) {
                 const int b = t / p.mtiles;
+                // Resident mode (the ring holds every tile of a batch element: stage j = tile j):
+                // the tiles are loaded again only when the batch element changes; otherwise the
+                // stage's phase just advances.
+                const bool reload = !p.resident || b != cur_b;
+                cur_b = b;
                 for (int j = 0; j < p.nct; ++j) {
                     const int crow = j * BN + static_cast<int>(rank) * CROWS;
                     if (!mbar_wait(C_EMPTY(stage), cph ^ 1u, abortp)) { ok = false; break; }
+                    if (!reload) {
+                        if (leader) mbar_arrive(C_FULL(stage));
+                        ++n_c;
+                        if (++stage == S) { stage = 0; cph ^= 1u; }
+                        continue;
+                    }
                     if (leader) mbar_arrive_expect_tx(C_FULL(stage), stage_tx);
                     const uint32_t sdst = sbase + L.c_off + stage * L.stage;
                     const uint32_t lbar = map_to_rank(C_FULL(stage), 0);
@@ -388,7 +411,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 }
             }
             if (!ok && leader) {
-                // Let every pair copy issued into the ring land before shared memory goes away.
+                // Let every pair copy issued into the ring land before shared memory goes away
+                // (n_c counts every use of the ring, so each stage's last phase is known).
                 for (int s = 0; s < S; ++s) {
                     const long long uses = n_c > s ? (n_c - 1 - s) / S + 1 : 0;
                     if (uses) mbar_wait(C_FULL(s), static_cast<uint32_t>((uses - 1) & 1), nullptr);
@@ -397,118 +421,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         }
         __syncwarp();
     } else if (warp == WARP_XPROD) {
-        // ------------------------------------------------------------ point producer
-        if (lane == 0) {
-            const uint64_t pol_x = l2_policy_evict_first();
-            int n_x = 0;
-            bool ok = true;
-            int local = 0;
-            for (int t = cluster_id; t < total; t += nclusters, ++local) {
-                const int b = t / p.mtiles;
-                const int m0 = (t % p.mtiles) * (2 * BM) + static_cast<int>(rank) * BM;
-                const int xb = local & 1;
-                const uint32_t xph = (local >> 1) & 1;
-                if (!mbar_wait(X_EMPTY(xb), xph ^ 1u, abortp)) { ok = false; break; }
+        // ------------------------------------------------------------ point tiles and norms
+        const uint64_t pol_x = l2_policy_evict_first();
+        float *dbuf = reinterpret_cast<float *>(sgen + L.delta_off);
+        const uint32_t xaug_full_leader0 = map_to_rank(XAUG_FULL(0), 0);
+        const uint32_t xaug_full_leader1 = map_to_rank(XAUG_FULL(1), 0);
+        int n_x = 0;
+        bool ok = true;
+        int local = 0;
+        for (int t = t_begin; t < t_end; ++t, ++local) {
+            const int b = t / p.mtiles;
+            const int m0 = (t % p.mtiles) * (2 * BM) + static_cast<int>(rank) * BM;
+            const int xb = local & 1;
+            const uint32_t xph = (local >> 1) & 1;
+            if (!mbar_wait_warp(X_EMPTY(xb), xph ^ 1u, abortp)) { ok = false; break; }
+            if (lane == 0) {
                 mbar_arrive_expect_tx(X_FULL(xb), NKC * XCHUNK);
                 for (int kc = 0; kc < NKC; ++kc)
                     tma_load_3d(sbase + L.x_off + (xb * NKC + kc) * XCHUNK, &tmX, X_FULL(xb),
                                 kc * KC, m0, b, pol_x);
-                ++n_x;
             }
-            if (!ok) {
-                for (int i = 0; i < 2; ++i) {
-                    const int uses = n_x > i ? (n_x - 1 - i) / 2 + 1 : 0;
-                    if (uses) mbar_wait(X_FULL(i), static_cast<uint32_t>((uses - 1) & 1), nullptr);
-                }
-            }
-        }
-        __syncwarp();
-    } else if (warp == WARP_MMA) {
-        // ------------------------------------------------------------ MMA issuer (leader)
-        if (leader) {
-            const bool issuer = elect_one();   // the same lane issues every MMA and commit
-            int stage = 0;
-            uint32_t cph = 0;
-            int abuf = 0;
-            uint32_t aph = 0;
-            int local = 0, j = 0;
-            int t = cluster_id;
-            bool ready = false;   // the current tile's barriers were already seen complete
-            const uint32_t cbase_lo = desc_lo(sbase + L.c_off);
-            const uint32_t xbase_lo = desc_lo(sbase + L.x_off);
-            const uint32_t xaug_lo = desc_lo(sbase + L.xaug_off);
-            const uint32_t stage16 = L.stage >> 4;
-            constexpr uint32_t cchunk16 = CCHUNK >> 4;
-            constexpr uint32_t xchunk16 = XCHUNK >> 4;
-            const int nk_last = (p.d - (NKC - 1) * KC + 15) / 16;   // K steps of the last chunk
-            while (t < total) {
-                const int xb = local & 1;
-                const uint32_t xph = (local >> 1) & 1;
-                if (!ready) {
-                    // both CTAs' point tiles landed and their augmentation rows are written; the
-                    // epilogue has read this accumulator; the centroid tile has landed
-                    if (j == 0 && !mbar_wait_warp(XAUG_FULL(xb), xph, abortp)) break;
-                    if (!mbar_wait_warp(ACC_EMPTY(abuf), aph ^ 1u, abortp)) break;
-                    if (!mbar_wait_warp(C_FULL(stage), cph, abortp)) break;
-                }
-                tc_fence_after();
-                const uint32_t dcol = tmem_base + abuf * ACC_STRIDE;
-                const uint32_t b_lo = cbase_lo + stage * stage16;
-                const uint32_t a_lo = xbase_lo + xb * (NKC * xchunk16);
-                if (issuer) {
-#pragma unroll
-                    for (int kc = 0; kc < NKC; ++kc)
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            if (kc + 1 < NKC || kk < nk_last)
-                                tc_mma_pair(dcol, a_lo + kc * xchunk16 + kk * 2, DESC_HI_SW128,
-                                            b_lo + kc * cchunk16 + kk * 2, DESC_HI_SW128,
-                                            p.idesc_main, (kc | kk) != 0 ? 1u : 0u);
-                }
-                __syncwarp();
-                // Next tile, and a look at its barriers while this tile's MMAs are queued.
-                int nj = j + 1, nlocal = local, nt = t;
-                if (nj == p.nct) { nj = 0; ++nlocal; nt += nclusters; }
-                const int nstage = stage + 1 == S ? 0 : stage + 1;
-                const uint32_t ncph = stage + 1 == S ? cph ^ 1u : cph;
-                const int nabuf = abuf ^ 1;
-                const uint32_t naph = abuf == 1 ? aph ^ 1u : aph;
-                bool nready = false;
-                if (nt < total) {
-                    nready = mbar_test_wait(ACC_EMPTY(nabuf), naph ^ 1u) &&
-                             mbar_test_wait(C_FULL(nstage), ncph) &&
-                             (nj != 0 || mbar_test_wait(XAUG_FULL(nlocal & 1), (nlocal >> 1) & 1));
-                }
-                ready = __shfl_sync(0xffffffffu, nready ? 1 : 0, 0) != 0;
-                if (issuer) {
-                    tc_mma_pair(dcol, xaug_lo + xb * (XAUG_BYTES >> 4), DESC_HI_SW32,
-                                b_lo + NKC * cchunk16, DESC_HI_SW32, p.idesc_aug, 1u);
-                    tc_commit_pair_both(ACC_FULL(abuf));
-                }
-                __syncwarp();
-                j = nj; local = nlocal; t = nt;
-                stage = nstage; cph = ncph; abuf = nabuf; aph = naph;
-            }
-            // Every MMA issued above completes before TMEM is released.
-            if (issuer) tc_commit_pair_self(DRAIN);
             __syncwarp();
-            mbar_wait_warp(DRAIN, 0, nullptr);
-        }
-        __syncwarp();
-    } else if (warp < WARP_EPI0) {
-        // ------------------------------------------------------------ norms (both CTAs)
-        const int nw = warp - WARP_NORM0;
-        float *dbuf = reinterpret_cast<float *>(sgen + L.delta_off);
-        const uint32_t xaug_full_leader0 = map_to_rank(XAUG_FULL(0), 0);
-        const uint32_t xaug_full_leader1 = map_to_rank(XAUG_FULL(1), 0);
-        int local = 0;
-        for (int t = cluster_id; t < total; t += nclusters, ++local) {
-            const int xb = local & 1;
-            const uint32_t xph = (local >> 1) & 1;
-            if (!mbar_wait_warp(X_FULL(xb), xph, abortp)) break;
+            ++n_x;
+            // The tile's norms as soon as it lands (this warp has nothing else to do until the
+            // next buffer is handed back at the end of the work item before this one).
+            if (!mbar_wait_warp(X_FULL(xb), xph, abortp)) { ok = false; break; }
 #pragma unroll 1
-            for (int rr = 0; rr < BM / (32 * NUM_NORM_WARPS); ++rr) {
-                const int row = nw * 32 + lane + rr * 32 * NUM_NORM_WARPS;
+            for (int rr = 0; rr < BM / 32; ++rr) {
+                const int row = lane + rr * 32;
                 const float half_xn =
                     0.5f * tile_row_sqnorm<T>(sgen + L.x_off + xb * NKC * XCHUNK, NKC, row);
                 const float x1 = __bfloat162float(__float2bfloat16_rn(half_xn));
@@ -532,6 +472,75 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 mbar_arrive(X_EMPTY(xb));
             }
         }
+        if (!ok && lane == 0) {
+            // Let every point copy issued land before shared memory goes away.
+            for (int i = 0; i < 2; ++i) {
+                const int uses = n_x > i ? (n_x - 1 - i) / 2 + 1 : 0;
+                if (uses) mbar_wait(X_FULL(i), static_cast<uint32_t>((uses - 1) & 1), nullptr);
+            }
+        }
+        __syncwarp();
+    } else if (warp == WARP_MMA || warp == WARP_MMA_ODD) {
+        // ------------------------------------------------------------ MMA issuers (leader)
+        if (leader) {
+            const int abuf = warp == WARP_MMA ? 0 : 1;   // this warp's accumulator and tiles
+            const bool issuer = elect_one();   // the same lane issues every MMA and commit
+            uint32_t aph = 0;
+            // tile sequence number g = local * nct + j; this warp takes g % 2 == abuf
+            int local = 0, j = abuf;
+            int t = t_begin;
+            while (j >= p.nct) { j -= p.nct; ++local; ++t; }
+            int g = abuf;
+            int xaug_local = -1;   // the work item whose point rows were last seen ready
+            const uint32_t cbase_lo = desc_lo(sbase + L.c_off);
+            const uint32_t xbase_lo = desc_lo(sbase + L.x_off);
+            const uint32_t xaug_lo = desc_lo(sbase + L.xaug_off);
+            const uint32_t stage16 = L.stage >> 4;
+            constexpr uint32_t cchunk16 = CCHUNK >> 4;
+            constexpr uint32_t xchunk16 = XCHUNK >> 4;
+            const int nk_last = (p.d - (NKC - 1) * KC + 15) / 16;   // K steps of the last chunk
+            while (t < t_end) {
+                const int xb = local & 1;
+                const uint32_t xph = (local >> 1) & 1;
+                const int stage = g % S;
+                const uint32_t cph = (g / S) & 1;
+                // both CTAs' point tiles landed and their augmentation rows are written; the
+                // epilogue has read this accumulator; the centroid tile has landed
+                if (xaug_local != local) {
+                    if (!mbar_wait_warp(XAUG_FULL(xb), xph, abortp)) break;
+                    xaug_local = local;
+                }
+                if (!mbar_wait_warp(ACC_EMPTY(abuf), aph ^ 1u, abortp)) break;
+                if (!mbar_wait_warp(C_FULL(stage), cph, abortp)) break;
+                tc_fence_after();
+                const uint32_t dcol = tmem_base + abuf * ACC_STRIDE;
+                const uint32_t b_lo = cbase_lo + stage * stage16;
+                const uint32_t a_lo = xbase_lo + xb * (NKC * xchunk16);
+                if (issuer) {
+#pragma unroll
+                    for (int kc = 0; kc < NKC; ++kc)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            if (kc + 1 < NKC || kk < nk_last)
+                                tc_mma_pair(dcol, a_lo + kc * xchunk16 + kk * 2, DESC_HI_SW128,
+                                            b_lo + kc * cchunk16 + kk * 2, DESC_HI_SW128,
+                                            p.idesc_main, (kc | kk) != 0 ? 1u : 0u);
+                    tc_mma_pair(dcol, xaug_lo + xb * (XAUG_BYTES >> 4), DESC_HI_SW32,
+                                b_lo + NKC * cchunk16, DESC_HI_SW32, p.idesc_aug, 1u);
+                    tc_commit_pair_both(ACC_FULL(abuf));
+                }
+                __syncwarp();
+                aph ^= 1u;
+                g += 2;
+                j += 2;
+                while (j >= p.nct) { j -= p.nct; ++local; ++t; }
+            }
+            // Every MMA issued above completes before TMEM is released.
+            if (issuer) tc_commit_pair_self(DRAIN);
+            __syncwarp();
+            mbar_wait_warp(DRAIN, 0, nullptr);
+        }
+        __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int ew = warp - WARP_EPI0;
@@ -548,7 +557,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         uint32_t aph = 0;
         int stage = 0;
         int local = 0;
-        for (int t = cluster_id; t < total; t += nclusters, ++local) {
+        for (int t = t_begin; t < t_end; ++t, ++local) {
             const int b = t / p.mtiles;
             const int m0 = (t % p.mtiles) * (2 * BM) + static_cast<int>(rank) * BM;
             const int xb = local & 1;

@@ -223,7 +223,15 @@ template <typename T, int BN, int NKC>
 km_status launch_assign_tc(const CUtensorMap &tmX, const CUtensorMap &tmC, const CUtensorMap &tmA,
                            km::tc::Params &p, int64_t items, cudaStream_t st) {
     using namespace km::tc;
-    p.stages = pick_stages(NKC, BN);
+    // Keep every centroid tile of a batch element resident when the ring can hold them all
+    // (one reload per batch element instead of one per work item); else stream them.
+    if (p.nct >= 2 && p.nct <= MAX_STAGES && make_layout(NKC, BN, p.nct).total + 1024u <= SMEM_ATTR) {
+        p.stages = p.nct;
+        p.resident = 1;
+    } else {
+        p.stages = pick_stages(NKC, BN);
+        p.resident = 0;
+    }
     if (p.stages < 2) return KM_ERR_UNSUPPORTED;
     const Layout L = make_layout(NKC, BN, p.stages);
     // More than half of the shared memory per block keeps one CTA per SM, so no second CTA
@@ -326,6 +334,7 @@ km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float 
     p.nct = static_cast<int>(Kp / bn);
     p.mtiles = static_cast<int>(ceil_div(N, 2 * BM));   // 256-point items, one per SM pair
     p.stages = 2;
+    p.resident = 0;
     p.need_dist = (mind || inertia) ? 1 : 0;
     // M = 256 across the pair; main step with A (the points) negated, so the accumulator
     // collects -<x, c>
