@@ -63,6 +63,8 @@ def _load():
         "km_assign_uses_tensor_cores": ([I, I64, P, P], I),
         "km_update_noalloc": ([P, I, P, P, I64, I64, I64, I64, P, P, P, P, P], I),
         "km_noalloc_scratch_needed": ([I64, I64, I64, I64], SZ),
+        "km_stream_workspace_size": ([I64, I64, I64, I, I, I64], SZ),
+        "km_fit_stream": ([P, I, P, I64, I64, I64, I64, P, I, I64, P, P, SZ, P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -262,6 +264,28 @@ def km_fit_host(X_host, C_host, iters, w_host=None, ids_host=None, inertia_host=
         _p(X_host), _dt(X_host.dtype), _p(w_host), B, N, K, d, _p(C_host), iters, _p(ids_host),
         _p(inertia_host), _p(ws), ws.numel(), _s(stream)))
     return C_host
+
+
+def km_fit_stream(X_host, C, iters, chunk, w_host=None, want_inertia=False, ws=None, stream=None):
+    """Out-of-core fit: X_host [B,N,d] (host, pinned for overlap) streamed in chunks of `chunk`
+    points per batch element every iteration; C [B,K,d] fp32 on the device, updated in place.
+    Returns (C, inertia_hist [iters,B] fp64 on the device, or None). Asynchronous on `stream`."""
+    B, N, d = X_host.shape
+    K = C.shape[1]
+    dev = C.device
+    for t, n in ((X_host, "X_host"), (w_host, "w_host")):
+        if t is not None and (t.device.type != "cpu" or not t.is_contiguous()):
+            raise ValueError(f"{n} must be a contiguous host tensor")
+    _need(C, "C", torch.float32, (B, K, d))
+    inertia = torch.empty((iters, B), dtype=torch.float64, device=dev) if want_inertia and iters else None
+    if ws is None:
+        n = _load().km_stream_workspace_size(B, K, d, _dt(X_host.dtype), int(w_host is not None),
+                                             min(chunk, N))
+        ws = torch.empty(max(int(n), 1), dtype=torch.uint8, device=dev)
+    _check("km_fit_stream", _load().km_fit_stream(
+        _p(X_host), _dt(X_host.dtype), _p(w_host), B, N, K, d, _p(C), iters, chunk, _p(inertia),
+        _p(ws), ws.numel(), _s(stream)))
+    return C, inertia
 
 
 def km_assign_uses_tensor_cores(X, Cx):

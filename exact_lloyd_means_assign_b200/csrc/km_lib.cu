@@ -127,6 +127,36 @@ inline HostWs carve_host(Carver &c, int64_t B, int64_t N, int64_t K, int64_t d, 
     return h;
 }
 
+// Streamed fit: two device buffers of `chunk` points per batch element (X and weights), the
+// running per-cluster statistics, one chunk's sort and assignment scratch.
+struct StreamWs {
+    void *xbuf[2];
+    float *wbuf[2];
+    void *Cx;
+    float *cn;
+    int32_t *ids, *counts, *chunk_counts;
+    void *rest;   // UpdateWs for one chunk, then (reusing it) the assignment scratch
+};
+inline StreamWs carve_stream(Carver &c, int64_t B, int64_t K, int64_t d, km_dtype dt, bool weighted,
+                             int64_t chunk) {
+    StreamWs s;
+    for (int i = 0; i < 2; ++i) {
+        s.xbuf[i] = c.take<uint8_t>(static_cast<size_t>(B * chunk * d) * dtype_size(dt));
+        s.wbuf[i] = weighted ? c.take<float>(static_cast<size_t>(B * chunk) * 4) : nullptr;
+    }
+    s.Cx = c.take<uint8_t>(static_cast<size_t>(B * K * d) * dtype_size(dt));
+    s.cn = c.take<float>(static_cast<size_t>(B * K) * 4);
+    s.ids = c.take<int32_t>(static_cast<size_t>(B * chunk) * 4);
+    s.counts = c.take<int32_t>(static_cast<size_t>(B * K) * 4);
+    s.chunk_counts = c.take<int32_t>(static_cast<size_t>(B * K) * 4);
+    s.rest = c.base ? c.base + c.off : nullptr;
+    Carver u(nullptr);
+    carve_update(u, B, chunk, K, d);
+    c.off += u.off;   // the running sums/wsum live in this UpdateWs; the assignment scratch follows
+    c.off += align_up(ws_assign(B, K, d, dt));
+    return s;
+}
+
 // ---------------------------------------------------------------- device queries
 
 int num_sms() {
@@ -359,10 +389,13 @@ km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float 
 
 // Validated-argument assignment; `caug` must hold ws_assign(B, K, d) bytes when the tensor-core
 // path can run.
+// With accumulate_inertia the objective is added to `inertia` instead of overwriting it (the
+// streamed fit sums it over chunks of points).
 km_status do_assign(const void *X, km_dtype dt, const void *Cx, const float *cn, const float *w,
                     int64_t B, int64_t N, int64_t K, int64_t d, int32_t *ids, float *mind,
-                    double *inertia, void *caug, cudaStream_t st) {
-    if (inertia && cudaMemsetAsync(inertia, 0, static_cast<size_t>(B) * 8, st) != cudaSuccess)
+                    double *inertia, void *caug, cudaStream_t st, bool accumulate_inertia = false) {
+    if (inertia && !accumulate_inertia &&
+        cudaMemsetAsync(inertia, 0, static_cast<size_t>(B) * 8, st) != cudaSuccess)
         return KM_ERR_CUDA;
     const bool tc = tc_shape_ok(dt, d) && aligned(X, 16) && aligned(Cx, 16) && caug != nullptr &&
                     B * ceil_div(N, 128) <= kMaxIndex;
@@ -491,13 +524,23 @@ km_status segreduce_dispatch(const void *X, const float *w, const int32_t *perm,
 }
 
 // sums[B,K,d], counts[B,K] and (when non-null) wsum[B,K] are overwritten.
+// Accumulating form (sort_counts != nullptr): sums, wsum and counts are added to, not
+// overwritten; the sort of this call's points uses `sort_counts` (B*K int32 scratch), which is
+// then added into `counts`.
 km_status do_update_partial(const void *X, km_dtype dt, const int32_t *ids, const float *w,
                             int64_t B, int64_t N, int64_t K, int64_t d, float *sums, float *wsum,
-                            int32_t *counts, const UpdateWs &u, cudaStream_t st) {
-    if (cudaMemsetAsync(counts, 0, static_cast<size_t>(B * K) * 4, st) != cudaSuccess ||
-        cudaMemsetAsync(sums, 0, static_cast<size_t>(B * K * d) * 4, st) != cudaSuccess ||
-        (wsum && cudaMemsetAsync(wsum, 0, static_cast<size_t>(B * K) * 4, st) != cudaSuccess))
+                            int32_t *counts, const UpdateWs &u, cudaStream_t st,
+                            int32_t *sort_counts = nullptr) {
+    int32_t *total_counts = counts;
+    if (sort_counts) {
+        counts = sort_counts;
+        if (cudaMemsetAsync(counts, 0, static_cast<size_t>(B * K) * 4, st) != cudaSuccess)
+            return KM_ERR_CUDA;
+    } else if (cudaMemsetAsync(counts, 0, static_cast<size_t>(B * K) * 4, st) != cudaSuccess ||
+               cudaMemsetAsync(sums, 0, static_cast<size_t>(B * K * d) * 4, st) != cudaSuccess ||
+               (wsum && cudaMemsetAsync(wsum, 0, static_cast<size_t>(B * K) * 4, st) != cudaSuccess)) {
         return KM_ERR_CUDA;
+    }
     using namespace km::upd;
     const bool smem_bins = K <= SMEM_K_MAX;
     const int64_t ntiles = ceil_div(N, TILE);
@@ -526,12 +569,15 @@ km_status do_update_partial(const void *X, km_dtype dt, const int32_t *ids, cons
             u.perm + b0 * N, smem_bins);
         if (launch_status() != KM_OK) return KM_ERR_CUDA;
     }
+    km_status s;
     switch (dt) {
-        case KM_F32: return segreduce_dispatch<float>(X, w, u.perm, u.offsets, B, N, K, d, sums, wsum, st);
-        case KM_F16: return segreduce_dispatch<__half>(X, w, u.perm, u.offsets, B, N, K, d, sums, wsum, st);
-        default:
-            return segreduce_dispatch<__nv_bfloat16>(X, w, u.perm, u.offsets, B, N, K, d, sums, wsum, st);
+        case KM_F32: s = segreduce_dispatch<float>(X, w, u.perm, u.offsets, B, N, K, d, sums, wsum, st); break;
+        case KM_F16: s = segreduce_dispatch<__half>(X, w, u.perm, u.offsets, B, N, K, d, sums, wsum, st); break;
+        default: s = segreduce_dispatch<__nv_bfloat16>(X, w, u.perm, u.offsets, B, N, K, d, sums, wsum, st);
     }
+    if (s != KM_OK || !sort_counts) return s;
+    add_i32_kernel<<<static_cast<unsigned>(ceil_div(B * K, 256)), 256, 0, st>>>(total_counts, sort_counts, B * K);
+    return launch_status();
 }
 
 template <typename T>
@@ -592,6 +638,86 @@ km_status do_fit(const void *X, km_dtype dt, const float *w, int64_t B, int64_t 
 }
 
 inline bool elem_aligned(const void *p, km_dtype dt) { return aligned(p, dtype_size(dt)); }
+
+// Out-of-core Lloyd: every iteration streams X (and w) from host memory through two device
+// buffers of `chunk` points per batch element. Copies run on their own stream; chunk c's
+// assignment and accumulation wait for its copy, and the copy into a buffer waits until the
+// chunk that last used it has been processed, so copy c+1 overlaps compute c.
+km_status do_fit_stream(const void *Xh, km_dtype dt, const float *wh, int64_t B, int64_t N,
+                        int64_t K, int64_t d, float *C, int iters, int64_t chunk,
+                        double *inertia_hist, void *ws, cudaStream_t st) {
+    Carver c(ws);
+    StreamWs sw = carve_stream(c, B, K, d, dt, wh != nullptr, chunk);
+    Carver r(sw.rest);
+    UpdateWs u = carve_update(r, B, chunk, K, d);
+    void *caug = r.base + r.off;
+    const size_t esz = dtype_size(dt);
+    const int64_t nch = ceil_div(N, chunk);
+    cudaStream_t cp = nullptr;
+    cudaEvent_t ready[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
+    km_status s = KM_OK;
+    auto cleanup = [&]() {   // resources are released once the enqueued work has finished
+        for (int i = 0; i < 2; ++i) {
+            if (ready[i]) cudaEventDestroy(ready[i]);
+            if (freed[i]) cudaEventDestroy(freed[i]);
+        }
+        if (cp) cudaStreamDestroy(cp);
+    };
+    if (cudaStreamCreateWithFlags(&cp, cudaStreamNonBlocking) != cudaSuccess) { cleanup(); return KM_ERR_CUDA; }
+    for (int i = 0; i < 2; ++i)
+        if (cudaEventCreateWithFlags(&ready[i], cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&freed[i], cudaEventDisableTiming) != cudaSuccess) {
+            cleanup();
+            return KM_ERR_CUDA;
+        }
+    // the copy stream starts after everything the caller enqueued before this call
+    if (cudaEventRecord(freed[0], st) != cudaSuccess || cudaStreamWaitEvent(cp, freed[0], 0) != cudaSuccess) {
+        cleanup();
+        return KM_ERR_CUDA;
+    }
+    s = prep_dispatch(C, dt, B * K, d, sw.Cx, sw.cn, st);
+    bool used[2] = {false, false};
+    for (int t = 0; t < iters && s == KM_OK; ++t) {
+        double *in = inertia_hist ? inertia_hist + static_cast<int64_t>(t) * B : nullptr;
+        if (cudaMemsetAsync(sw.counts, 0, static_cast<size_t>(B * K) * 4, st) != cudaSuccess ||
+            cudaMemsetAsync(u.sums, 0, static_cast<size_t>(B * K * d) * 4, st) != cudaSuccess ||
+            (wh && cudaMemsetAsync(u.wsum, 0, static_cast<size_t>(B * K) * 4, st) != cudaSuccess) ||
+            (in && cudaMemsetAsync(in, 0, static_cast<size_t>(B) * 8, st) != cudaSuccess)) {
+            s = KM_ERR_CUDA;
+            break;
+        }
+        for (int64_t ch = 0; ch < nch && s == KM_OK; ++ch) {
+            const int i = static_cast<int>(ch & 1);
+            const int64_t n0 = ch * chunk, n = std::min(chunk, N - n0);
+            if (used[i] && cudaStreamWaitEvent(cp, freed[i], 0) != cudaSuccess) { s = KM_ERR_CUDA; break; }
+            // rows n0..n0+n of every batch element: one 2-D copy (B rows of n * d elements)
+            if (cudaMemcpy2DAsync(sw.xbuf[i], static_cast<size_t>(n * d) * esz,
+                                  static_cast<const uint8_t *>(Xh) + static_cast<size_t>(n0 * d) * esz,
+                                  static_cast<size_t>(N * d) * esz, static_cast<size_t>(n * d) * esz,
+                                  static_cast<size_t>(B), cudaMemcpyHostToDevice, cp) != cudaSuccess ||
+                (wh && cudaMemcpy2DAsync(sw.wbuf[i], static_cast<size_t>(n) * 4, wh + n0,
+                                         static_cast<size_t>(N) * 4, static_cast<size_t>(n) * 4,
+                                         static_cast<size_t>(B), cudaMemcpyHostToDevice, cp) != cudaSuccess) ||
+                cudaEventRecord(ready[i], cp) != cudaSuccess || cudaStreamWaitEvent(st, ready[i], 0) != cudaSuccess) {
+                s = KM_ERR_CUDA;
+                break;
+            }
+            s = do_assign(sw.xbuf[i], dt, sw.Cx, sw.cn, sw.wbuf[i], B, n, K, d, sw.ids, nullptr, in,
+                          caug, st, true);
+            if (s != KM_OK) break;
+            s = do_update_partial(sw.xbuf[i], dt, sw.ids, sw.wbuf[i], B, n, K, d, u.sums,
+                                  wh ? u.wsum : nullptr, sw.counts, u, st, sw.chunk_counts);
+            if (s != KM_OK) break;
+            if (cudaEventRecord(freed[i], st) != cudaSuccess) { s = KM_ERR_CUDA; break; }
+            used[i] = true;
+        }
+        if (s == KM_OK)
+            s = finalize_dispatch(u.sums, wh ? u.wsum : nullptr, sw.counts, C, B * K, d, C, dt, sw.Cx,
+                                  sw.cn, st);
+    }
+    cleanup();
+    return s;
+}
 
 }  // namespace
 
@@ -732,6 +858,28 @@ km_status km_fit(const void *X, km_dtype dtype, const float *w, int64_t B, int64
         if (!ws || ws_bytes < c.off || !aligned(ws, kAlign)) return KM_ERR_WORKSPACE;
     }
     return do_fit(X, dtype, w, B, N, K, d, C, iters, ids, inertia_hist, C_hist, ws, S(stream));
+}
+
+size_t km_stream_workspace_size(int64_t B, int64_t K, int64_t d, km_dtype dtype, int weighted,
+                                int64_t chunk) {
+    if (!sizes_ok(B, chunk, K, d) || !valid_dtype(dtype)) return 0;
+    Carver c(nullptr);
+    carve_stream(c, B, K, d, dtype, weighted != 0, chunk);
+    return c.off;
+}
+
+km_status km_fit_stream(const void *X_host, km_dtype dtype, const float *w_host, int64_t B,
+                        int64_t N, int64_t K, int64_t d, float *C, int iters, int64_t chunk,
+                        double *inertia_hist, void *ws, size_t ws_bytes, void *stream) {
+    if (!X_host || !C || iters < 0 || !valid_dtype(dtype) || !sizes_ok(B, N, K, d) || chunk < 1 ||
+        !aligned(C, 4) || (inertia_hist && !aligned(inertia_hist, 8)) ||
+        !aligned(X_host, dtype_size(dtype)) || (w_host && !aligned(w_host, 4)))
+        return KM_ERR_INVALID_ARG;
+    chunk = std::min(chunk, N);
+    if (!ws || ws_bytes < km_stream_workspace_size(B, K, d, dtype, w_host != nullptr, chunk) ||
+        !aligned(ws, kAlign))
+        return KM_ERR_WORKSPACE;
+    return do_fit_stream(X_host, dtype, w_host, B, N, K, d, C, iters, chunk, inertia_hist, ws, S(stream));
 }
 
 km_status km_fit_host(const void *X_host, km_dtype dtype, const float *w_host, int64_t B,

@@ -156,6 +156,12 @@ __global__ void __launch_bounds__(TILE_THREADS)
     }
 }
 
+// dst[i] += src[i] (per-cluster counts of one chunk of points added to the running counts)
+__global__ void add_i32_kernel(int32_t *__restrict__ dst, const int32_t *__restrict__ src, int64_t n) {
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i < n) dst[i] += src[i];
+}
+
 template <typename T, int VEC> struct alignas(sizeof(T) * VEC) VecT {
     T v[VEC];
 };

@@ -1,7 +1,9 @@
 """Multi-GPU Lloyd iterations: one process per GPU, ``torch.distributed`` for the exchange.
 
-Two ways the iteration splits over ranks (wispaper blog "Distributed and large-scale
-settings"; Flash-KMeans article, exact Lloyd per iteration):
+The pages describe a single-GPU method; how it splits over ranks follows from the iteration
+itself (the Lloyd recap in the technologypulse.uk Flash-KMeans article and the steinslab e-means
+daily: the assignment is independent per point and the update is a per-cluster sum divided by a
+count). Two ways:
 
 * Batch sharding. Every batch element is an independent k-means problem, so each rank owns a
   contiguous range of whole problems and runs the full iteration on it. There is no exchange

@@ -183,6 +183,30 @@ km_status km_fit_host(const void *X_host, km_dtype dtype, const float *w_host, i
                       int64_t N, int64_t K, int64_t d, float *C_host, int iters, int32_t *ids_host,
                       double *inertia_host, void *ws, size_t ws_bytes, void *stream);
 
+/* Out-of-core exact Lloyd (technologypulse.uk Flash-KMeans article, the out-of-core line of the
+ * measurements and the chunked stream overlap that hides PCIe transfers; wispaper blog
+ * "Performance", the scalability point): points that do not fit in device memory stay in
+ * host memory and are streamed through the GPU every iteration in chunks; each chunk is
+ * assigned as it arrives and its per-cluster sums and counts are accumulated, so the result is
+ * the exact Lloyd iteration of the whole set (up to fp32 summation order).
+ *   X_host[B,N,d] in host memory (pinned memory lets the copies overlap the kernels; pageable
+ *   memory works but the copies then block the calling thread), w_host[B,N] or NULL;
+ *   C[B,K,d] fp32 DEVICE memory: initial centroids in, final centroids out;
+ *   iters >= 0; chunk >= 1 points per batch element per copy (clamped to N);
+ *   inertia_hist[iters,B] fp64 DEVICE memory or NULL: the objective of each iteration's
+ *   assignment. Two device buffers of `chunk` points per batch element; copies run on a stream
+ *   the call creates and releases, ordered after the work already enqueued on `stream`.
+ *   Asynchronous on `stream` like km_fit; X_host and w_host must stay valid and unchanged until
+ *   the stream has completed the call's work.
+ * Errors: KM_ERR_INVALID_ARG (null pointers, sizes, chunk < 1, misaligned), KM_ERR_WORKSPACE
+ * (ws smaller than km_stream_workspace_size), KM_ERR_CUDA.
+ */
+size_t km_stream_workspace_size(int64_t B, int64_t K, int64_t d, km_dtype dtype, int weighted,
+                                int64_t chunk);
+km_status km_fit_stream(const void *X_host, km_dtype dtype, const float *w_host, int64_t B,
+                        int64_t N, int64_t K, int64_t d, float *C, int iters, int64_t chunk,
+                        double *inertia_hist, void *ws, size_t ws_bytes, void *stream);
+
 /*
  * Synchronises `stream`, then reads and clears the device error word of the current device.
  * *code = 0 when no kernel recorded an error; otherwise a bit mask (1 = a bounded wait ran out).

@@ -69,6 +69,12 @@ def test_workspace_sizes(lib):
     assert host >= fit + 32 * 65536 * 128 * 2 + 32 * 65536 * 4
     for bad in [(0, 1, 1, 1), (1, 0, 1, 1), (1, 1, 0, 1), (1, 1, 1, 0), (1, 1 << 31, 1, 1)]:
         assert km.km_workspace_size(km.KM_OP_UPDATE, *bad, f16) == 0
+    # streamed fit: scratch grows with the chunk, not with N; two chunk buffers of points
+    s1 = lib.km_stream_workspace_size(32, 1024, 128, 1, 0, 4096)
+    s2 = lib.km_stream_workspace_size(32, 1024, 128, 1, 0, 8192)
+    assert 2 * 32 * 4096 * 128 * 2 <= s1 and s2 - s1 >= 2 * 32 * 4096 * 128 * 2
+    assert lib.km_stream_workspace_size(32, 1024, 128, 1, 1, 4096) >= s1 + 2 * 32 * 4096 * 4
+    assert lib.km_stream_workspace_size(32, 1024, 128, 1, 0, 0) == 0
     for op in range(4):
         assert km.km_workspace_size(op, 3, 1000, 17, 24, f16, True, 5) % 256 == 0
 
@@ -104,6 +110,10 @@ def test_argument_errors_return_before_any_launch(lib):
     assert lib.km_fit(fake, 1, null, 1, 10, 4, 8, fake, 3, null, null, null, null, 0, st) == 3
     # km_fit_host: null host pointers
     assert lib.km_fit_host(null, 1, null, 1, 10, 4, 8, fake, 3, null, null, fake, 1 << 30, st) == 1
+    # km_fit_stream: null host X, chunk < 1, and a workspace smaller than the chunked scratch
+    assert lib.km_fit_stream(null, 1, null, 1, 10, 4, 8, fake, 3, 4, null, fake, 1 << 30, st) == 1
+    assert lib.km_fit_stream(fake, 1, null, 1, 10, 4, 8, fake, 3, 0, null, fake, 1 << 30, st) == 1
+    assert lib.km_fit_stream(fake, 1, null, 1, 10, 4, 8, fake, 3, 4, null, fake, 16, st) == 3
     # km_init_grid1d: d is implied 1, K must be >= 1
     assert lib.km_init_grid1d(fake, 1, 1, 10, 0, fake, st) == 1
     # km_prep: nothing to write

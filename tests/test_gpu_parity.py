@@ -278,6 +278,66 @@ def test_fit_host_matches_device(cuda_device):
     assert (idsh.numpy() != to_np(ids)).mean() < 1e-3
 
 
+STREAM_CASES = {
+    # (dtype, B, N, K, d, chunk, weighted): ragged last chunk, several tiles per chunk
+    "f16_tc": (torch.float16, 2, 5000, 300, 128, 1536, False),
+    "f32_exact_weighted": (torch.float32, 3, 3000, 64, 32, 700, True),
+    "bf16_one_chunk": (torch.bfloat16, 1, 2500, 130, 64, 4096, True),
+}
+
+
+@pytest.mark.parametrize("case", list(STREAM_CASES))
+def test_fit_stream_per_iteration(case, cuda_device):
+    dtype, B, N, K, d, chunk, weighted = STREAM_CASES[case]
+    X, C = mixture(B, N, d, K, dtype, "cpu", seed=11)
+    g = torch.Generator().manual_seed(5)
+    w = torch.rand((B, N), generator=g) * 2 + 0.05 if weighted else None
+    Xh = X.pin_memory()
+    wh = None if w is None else w.pin_memory()
+    Xd = X.to(cuda_device)
+    wd = None if w is None else w.to(cuda_device)
+    X64 = oracle.as_f64(X)
+    w64 = None if w is None else oracle.as_f64(w)
+    Cd = C.to(cuda_device)
+    for t in range(3):
+        C_prev = Cd.clone()
+        _, ih = km.km_fit_stream(Xh, Cd, 1, chunk, w_host=wh, want_inertia=True)
+        torch.cuda.synchronize()
+        Cp = to_np(C_prev).astype(np.float64)
+        ids_t, d1, d2, inertia = oracle.assign(X64, oracle.round_to_dtype(Cp, dtype), w64)
+        np.testing.assert_allclose(to_np(ih[0]), inertia, rtol=1e-4)
+        # the same assignment on the resident points (deterministic kernels): oracle ids
+        # except at near ties; the update of that assignment is the oracle's
+        Cx, cn = km.km_prep(C_prev, dtype)
+        ids_g, _, _ = km.km_assign(Xd, Cx, cn, w=wd)
+        torch.cuda.synchronize()
+        ig = to_np(ids_g)
+        assert not ((ig != ids_t) & ~oracle.near_tie(d1, d2)).any(), t
+        C_ref, _, _ = oracle.update(X64, ig.astype(np.int32), Cp, w64)
+        Cn = to_np(Cd).astype(np.float64)
+        for b in range(B):
+            err = np.linalg.norm(Cn[b] - C_ref[b]) / np.linalg.norm(C_ref[b])
+            assert err <= 1e-3, (t, b, err)
+
+
+def test_fit_stream_matches_resident_fit(cuda_device):
+    d = synth.make_workload(3, B=2, N=6000, K=256, device="cpu")
+    X, C0 = d["X"], d["C0"]
+    Cs = C0.to(cuda_device)
+    _, ih_s = km.km_fit_stream(X.pin_memory(), Cs, 4, 1000, want_inertia=True)
+    Cr = C0.to(cuda_device)
+    _, _, ih_r, _ = km.km_fit(X.to(cuda_device), Cr, 4, want_inertia=True)
+    torch.cuda.synchronize()
+    # only the order of the fp32 accumulation differs (per chunk, then across chunks)
+    torch.testing.assert_close(Cs, Cr, rtol=1e-4, atol=1e-5)
+    np.testing.assert_allclose(to_np(ih_s), to_np(ih_r), rtol=1e-5)
+    # zero iterations leave C untouched
+    C_keep = Cs.clone()
+    km.km_fit_stream(X.pin_memory(), Cs, 0, 1000)
+    torch.cuda.synchronize()
+    assert torch.equal(Cs, C_keep)
+
+
 def test_fit_k_greater_than_n_keeps_empty(cuda_device):
     X, C = mixture(1, 50, 32, 80, torch.float16, cuda_device, seed=9)
     C0 = C.clone()
