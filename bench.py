@@ -7,6 +7,7 @@ larger than the 126 MB L2, so no flush is needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
   python bench.py --out-of-core {batched_assign_bound,single_N33M_K16384} --steps 5
+  python bench.py --workload {tiny_exact,rows_weighted_1d,large_k_assign,contention_update}
 
 A step on the GPU = km_assign (tensor-core FlashAssign; the labels, which is all a Lloyd
 iteration needs: the per-point distance and the inertia are optional outputs) + km_update
@@ -337,6 +338,152 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def _timed(fn, steps, stream):
+    """Mean device ms of fn() over ``steps`` calls (CUDA events on ``stream``)."""
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        fn()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1) / steps
+
+
+def run_workload(args):
+    """The other synthetic workloads of the measurement table, one JSON line each, 1 GPU:
+    tiny_exact (latency, fp32 exact path, eager and CUDA-graph replay of a 20-iteration fit),
+    rows_weighted_1d (the fused per-row 1-D fit, K=16 and K=8, ALU roofline),
+    large_k_assign and contention_update (one Lloyd iteration per step: tensor-core roofline
+    for the assignment, HBM roofline for the sort-inverse update)."""
+    import exact_lloyd_means_assign_b200 as km
+    import synth
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    wl = synth.WORKLOADS[{w.name: i for i, w in synth.WORKLOADS.items()}[args.workload]]
+    peak_tf, peak_bw, peak_kind = _peaks()
+    base = {"n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "scaling": "none", "vs_baseline": None, "data": "synthetic",
+            "dtype": {torch.float32: "f32", torch.float16: "f16", torch.bfloat16: "bf16"}[wl.dtype]}
+    lines = []
+    if wl.name == "tiny_exact":
+        d = synth.make_workload(wl.idx, device=dev)
+        X, C0 = d["X"], d["C0"]
+        Bw, Nw, Dw = X.shape
+        Kw, iters = C0.shape[1], d["iters"]
+        ws = km.workspace(km.KM_OP_FIT, Bw, Nw, Kw, Dw, X.dtype, dev)
+        C = C0.clone()
+
+        def fit():   # on the current stream: the capture stream while the graph is recorded
+            C.copy_(C0)
+            km.km_fit(X, C, iters, ws=ws)
+
+        for _ in range(args.warmup):
+            fit()
+        with ClockSampler(0) as clk:
+            eager = _timed(fit, args.steps, stream)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fit()
+            graph = _timed(g.replay, args.steps, stream)
+        lines.append(dict(base, metric="exact fp32 Lloyd us/iteration (CUDA-core path)",
+                          value=graph * 1e3 / iters, unit="us/iter", higher_is_better=False,
+                          ms_per_step=graph,
+                          eager_us_per_iter=eager * 1e3 / iters,
+                          config={"workload": wl.name, "B": Bw, "N": Nw, "K": Kw, "d": Dw,
+                                  "iterations_per_step": iters, "launch": "CUDA graph of one km_fit call"},
+                          roofline={"bound": "latency", "note": "4.2 MFLOP per iteration; launch-bound"},
+                          clocks=clk.summary()))
+    elif wl.name == "rows_weighted_1d":
+        for Kw in wl.K:
+            d = synth.make_workload(wl.idx, device=dev, K=Kw)
+            X, w = d["X"], d["w"]
+            Bw, Nw = X.shape[0], X.shape[1]
+            iters = d["iters"]
+            C = torch.empty((Bw, Kw, 1), dtype=torch.float32, device=dev)
+
+            def fit():
+                km.km_init_grid1d(X, Kw, C=C, stream=stream)
+                km.km_fit(X, C, iters, w=w, stream=stream)
+
+            for _ in range(args.warmup):
+                fit()
+            with ClockSampler(0) as clk:
+                ms = _timed(fit, args.steps, stream)
+            clocks = clk.summary()
+            # peak: 128 fp32 lanes per SM per clock x SMs x the median SM clock under load
+            mhz = clocks.get("sm_mhz") or 1965.0
+            alu_peak = 128 * torch.cuda.get_device_properties(dev).multi_processor_count * mhz * 1e6 / 1e12
+            ops = 3.0 * Bw * Nw * Kw * iters   # brute-force equivalent: sub, mul, min per pair
+            lines.append(dict(base, metric="weighted 1-D per-row fit iter/s (all rows)",
+                              value=iters * 1e3 / ms, unit="iter/s", ms_per_step=ms,
+                              config={"workload": wl.name, "B": Bw, "N": Nw, "K": Kw, "d": 1,
+                                      "iterations_per_step": iters, "weighted": True, "init": "grid"},
+                              roofline={"bound": "alu", "achieved": ops / (ms * 1e-3) / 1e12,
+                                        "peak": alu_peak, "unit": "Tops/s",
+                                        "frac": ops / (ms * 1e-3) / 1e12 / alu_peak,
+                                        "note": "achieved counts 3 ops per (point, centroid) pair "
+                                                "(brute force); the kernel does fewer (sorted "
+                                                "centroids), so frac may exceed 1",
+                                        "peak_source": "128 fp32 lanes/SM/clk x SMs x median SM clock"},
+                              hbm_bytes_per_fit=Bw * Nw * (X.element_size() + 4),
+                              clocks=clocks))
+    else:
+        d = synth.make_workload(wl.idx, device=dev)
+        X, C = d["X"], d["C0"]
+        Bw, Nw, Dw = X.shape
+        Kw = C.shape[1]
+        ws_a = km.workspace(km.KM_OP_ASSIGN, Bw, Nw, Kw, Dw, X.dtype, dev)
+        ws_u = km.workspace(km.KM_OP_UPDATE, Bw, Nw, Kw, Dw, X.dtype, dev)
+        ids = torch.empty((Bw, Nw), dtype=torch.int32, device=dev)
+        counts = torch.empty((Bw, Kw), dtype=torch.int32, device=dev)
+        Cx, cn = km.km_prep(C, X.dtype)
+
+        def assign():
+            km.km_assign(X, Cx, cn, ids=ids, ws=ws_a, stream=stream)
+
+        def update():
+            km.km_update(X, ids, C, C_new=C, counts=counts, ws=ws_u, stream=stream)
+            km.km_prep(C, X.dtype, Cx=Cx, cn=cn, stream=stream)
+
+        for _ in range(args.warmup):
+            assign()
+            update()
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        with ClockSampler(0) as clk:
+            for e in ev:
+                e[0].record(stream)
+                assign()
+                e[1].record(stream)
+                update()
+                e[2].record(stream)
+            torch.cuda.synchronize()
+        a_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+        u_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+        flop = 2.0 * Bw * Nw * Kw * Dw
+        ubytes = Bw * Nw * Dw * X.element_size() + 4 * Bw * Nw * 4 + Bw * Kw * Dw * 4 * 2
+        line = dict(base, metric="Lloyd iter/s & assign pt·K/s; % roofline", value=1e3 / (a_ms + u_ms),
+                    unit="iter/s", ms_per_step=a_ms + u_ms, assign_ms=a_ms, update_ms=u_ms,
+                    assign_pt_k_per_s=Bw * Nw * Kw / (a_ms * 1e-3),
+                    config={"workload": wl.name, "B": Bw, "N": Nw, "K": Kw, "d": Dw,
+                            "iterations_per_step": 1, "l2": "inputs larger than L2"},
+                    roofline={"bound": "tensor", "kernel": "assign_tc_kernel",
+                              "achieved": flop / (a_ms * 1e-3) / 1e12, "peak": peak_tf,
+                              "unit": "TFLOP/s", "frac": flop / (a_ms * 1e-3) / 1e12 / peak_tf,
+                              "traffic": None, "peak_source": f"{peak_kind} bf16 dense"},
+                    update_roofline={"bound": "hbm", "achieved": ubytes / (u_ms * 1e-3) / 1e9,
+                                     "peak": peak_bw, "unit": "GB/s",
+                                     "frac": ubytes / (u_ms * 1e-3) / 1e9 / peak_bw,
+                                     "algorithmic_bytes": ubytes, "peak_source": peak_kind},
+                    gpu_launches=LAUNCHES_PER_STEP * args.steps, clocks=clk.summary(),
+                    device_error=km.km_device_error())
+        lines.append(line)
+    for l in lines:
+        print(json.dumps(l), flush=True)
+
+
 OOC_WORKLOADS = {
     # name: (synth workload, K override, points per batch element per chunk)
     "batched_assign_bound": (3, None, 16384),
@@ -409,11 +556,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--out-of-core", choices=sorted(OOC_WORKLOADS), default=None,
                     help="time the streamed fit (points in host memory) instead of the step")
+    ap.add_argument("--workload", default=None,
+                    choices=["tiny_exact", "rows_weighted_1d", "large_k_assign", "contention_update"],
+                    help="time one of the other synthetic workloads instead of the headline one")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.out_of_core:
         run_out_of_core(args)
+    elif args.workload:
+        run_workload(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

@@ -85,6 +85,29 @@ __device__ __forceinline__ int nearest(float x, const float *cx, int K) {
     return bi;
 }
 
+// Block-wide bitonic sort of NP (a power of two) (value, index) pairs in shared memory, ascending
+// by value; padding entries carry +inf. Ends with the block synchronised.
+__device__ __forceinline__ void sort_pairs_smem(float *xs, int *is, int NP) {
+    for (int k = 2; k <= NP; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int t = threadIdx.x; t < (NP >> 1); t += blockDim.x) {
+                const int i = 2 * j * (t / j) + (t % j);
+                const int ixj = i + j;
+                const bool asc = (i & k) == 0;
+                const float a = xs[i], c = xs[ixj];
+                if ((a > c) == asc) {
+                    xs[i] = c;
+                    xs[ixj] = a;
+                    const int ti = is[i];
+                    is[i] = is[ixj];
+                    is[ixj] = ti;
+                }
+            }
+            __syncthreads();
+        }
+    }
+}
+
 // Shared memory: NP floats (sorted values), NP ints (original index), NP floats (weights).
 template <typename T>
 __global__ void __launch_bounds__(THREADS)
@@ -115,25 +138,7 @@ __global__ void __launch_bounds__(THREADS)
     }
     __syncthreads();
 
-    // bitonic sort of (value, index) pairs, ascending
-    for (int k = 2; k <= NP; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int t = tid; t < (NP >> 1); t += THREADS) {
-                const int i = 2 * j * (t / j) + (t % j);
-                const int ixj = i + j;
-                const bool asc = (i & k) == 0;
-                const float a = xs[i], c = xs[ixj];
-                if ((a > c) == asc) {
-                    xs[i] = c;
-                    xs[ixj] = a;
-                    const int ti = is[i];
-                    is[i] = is[ixj];
-                    is[ixj] = ti;
-                }
-            }
-            __syncthreads();
-        }
-    }
+    sort_pairs_smem(xs, is, NP);
     for (int p = tid; p < N; p += THREADS)
         ws[p] = w ? w[static_cast<int64_t>(b) * N + is[p]] : 1.f;
     __syncthreads();
@@ -221,6 +226,315 @@ __global__ void __launch_bounds__(THREADS)
         __syncthreads();
     }
     if (tid < K) C[static_cast<int64_t>(b) * K + tid] = cm[tid];
+}
+
+// ---------------------------------------------------------------------------------------------
+// Warp-per-row form (K <= 32), for many rows. The fused kernel above keeps a row on chip, so only
+// a few rows fit on an SM and every phase of an iteration waits on the slowest thread of its row;
+// with thousands of rows it is latency-bound. Here the per-row state that an iteration needs is
+// reduced once, up front, to arrays in device memory:
+//   fit1d_sort_kernel  (one CTA per row): the sorted values, their original indices and the
+//                      prefix sums P0 = sum w, P1 = sum w*x, P2 = sum w*x^2 over the sorted order
+//                      (fp64, P[0] = 0);
+//   fit1d_iter_kernel  (one warp per row, every row resident at once): per iteration the K - 1
+//                      cluster boundaries by binary search over the sorted values (the same
+//                      exact-argmin test as above), then each cluster's weight, weighted sum and
+//                      objective from two prefix-sum reads:
+//                        W = P0[e] - P0[s], S = P1[e] - P1[s],
+//                        sum w (x - c)^2 = (P2[e] - P2[s]) - 2 c S + c^2 W.
+// An iteration then costs O(K log N) per row, independent of how many points each cluster holds.
+constexpr int ITER_WARPS = 4;   // rows per block of the iteration kernel
+constexpr int ITER_KMAX = 32;   // one centroid per lane
+
+// Order-preserving unsigned keys of the stored values (finite inputs): flip every bit of a
+// negative value, set the sign bit of a non-negative one.
+template <typename T> struct SortKey;
+template <> struct SortKey<float> {
+    static constexpr int BITS = 32;
+    static __device__ __forceinline__ uint32_t key(float v) {
+        const uint32_t u = __float_as_uint(v);
+        return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    }
+    static __device__ __forceinline__ float value(uint32_t k) {
+        return __uint_as_float((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k);
+    }
+};
+template <typename H, int DUMMY> struct SortKey16 {
+    static constexpr int BITS = 16;
+    static __device__ __forceinline__ uint32_t key(uint32_t u) {
+        return (u & 0x8000u) ? (~u & 0xffffu) : (u | 0x8000u);
+    }
+    static __device__ __forceinline__ uint16_t raw(uint32_t k) {
+        return static_cast<uint16_t>((k & 0x8000u) ? (k ^ 0x8000u) : (~k & 0xffffu));
+    }
+};
+template <> struct SortKey<__half> : SortKey16<__half, 0> {
+    static __device__ __forceinline__ uint32_t key(__half v) { return SortKey16::key(__half_as_ushort(v)); }
+    static __device__ __forceinline__ float value(uint32_t k) { return __half2float(__ushort_as_half(raw(k))); }
+};
+template <> struct SortKey<__nv_bfloat16> : SortKey16<__nv_bfloat16, 0> {
+    static __device__ __forceinline__ uint32_t key(__nv_bfloat16 v) {
+        return SortKey16::key(__bfloat16_as_ushort(v));
+    }
+    static __device__ __forceinline__ float value(uint32_t k) {
+        return __bfloat162float(__ushort_as_bfloat16(raw(k)));
+    }
+};
+
+// Stable LSD radix sort of one row in shared memory, 8-bit digits (2 passes for 16-bit values, 4
+// for fp32), by the block's THREADS threads. Warp w owns the contiguous positions
+// [w * seg, (w + 1) * seg) and walks them 32 at a time: lanes holding the same digit find each
+// other with a match, take consecutive slots after the warp's running count for that digit, and
+// the lowest of them advances the count. A block-wide scan over (digit, warp) then turns the
+// per-warp counts into destinations. Equal keys keep their order, so ties stay in index order.
+// Padding positions carry the largest key and sort to the end. Result in (ka, ia).
+constexpr int RADIX_WARPS = THREADS / 32;
+constexpr int RADIX_MAX_ROUNDS = NMAX / RADIX_WARPS / 32;
+
+template <int BITS>
+__device__ __forceinline__ void radix_sort_row(uint32_t *ka, uint16_t *ia, uint32_t *kb, uint16_t *ib,
+                                               int (*hist)[256], int seg) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int rounds = seg >> 5;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int shift = 0; shift < BITS; shift += 8) {
+        for (int i = lane; i < 256; i += 32) hist[warp][i] = 0;
+        __syncwarp();
+        int local[RADIX_MAX_ROUNDS];
+#pragma unroll
+        for (int r = 0; r < RADIX_MAX_ROUNDS; ++r) {
+            if (r < rounds) {
+                const int pos = warp * seg + r * 32 + lane;
+                const int dg = (ka[pos] >> shift) & 255;
+                const unsigned m = __match_any_sync(0xffffffffu, dg);
+                const int base = hist[warp][dg];
+                local[r] = base + __popc(m & lt);
+                __syncwarp();
+                if ((m & lt) == 0) hist[warp][dg] = base + __popc(m);
+                __syncwarp();
+            }
+        }
+        __syncthreads();
+        // thread t = digit t: warp bases for this digit, then an exclusive scan over digits
+        {
+            int tot = 0;
+            for (int v = 0; v < RADIX_WARPS; ++v) tot += hist[v][tid];
+            int inc = tot;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += u;
+            }
+            __shared__ int wsum[RADIX_WARPS];
+            if (lane == 31) wsum[warp] = inc;
+            __syncthreads();
+            int run = inc - tot;
+            for (int v = 0; v < warp; ++v) run += wsum[v];
+            for (int v = 0; v < RADIX_WARPS; ++v) {
+                const int c = hist[v][tid];
+                hist[v][tid] = run;
+                run += c;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < RADIX_MAX_ROUNDS; ++r) {
+            if (r < rounds) {
+                const int pos = warp * seg + r * 32 + lane;
+                const uint32_t k = ka[pos];
+                const int dst = hist[warp][(k >> shift) & 255] + local[r];
+                kb[dst] = k;
+                ib[dst] = ia[pos];
+            }
+        }
+        __syncthreads();
+        uint32_t *tk = ka;
+        ka = kb;
+        kb = tk;
+        uint16_t *ti = ia;
+        ia = ib;
+        ib = ti;
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(THREADS)
+    fit1d_sort_kernel(const T *__restrict__ X, const float *__restrict__ w, int N, int NP,
+                      float *__restrict__ xs_out, int32_t *__restrict__ is_out,
+                      double *__restrict__ P0, double *__restrict__ P1, double *__restrict__ P2) {
+    // shared memory: two key buffers (uint32) and two index buffers (uint16) of NP = 8 * seg
+    extern __shared__ uint8_t sm[];
+    uint32_t *ka = reinterpret_cast<uint32_t *>(sm);
+    uint32_t *kb = ka + NP;
+    uint16_t *ia = reinterpret_cast<uint16_t *>(kb + NP);
+    uint16_t *ib = ia + NP;
+    __shared__ int hist[RADIX_WARPS][256];
+    __shared__ double wtot[3][THREADS / 32];
+    const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const T *xb = X + static_cast<int64_t>(b) * N;
+    for (int p = tid; p < NP; p += THREADS) {
+        ka[p] = p < N ? SortKey<T>::key(xb[p]) : 0xffffffffu;
+        ia[p] = static_cast<uint16_t>(p);
+    }
+    __syncthreads();
+    radix_sort_row<SortKey<T>::BITS>(ka, ia, kb, ib, hist, NP / RADIX_WARPS);
+    // an even number of passes leaves the result in (ka, ia)
+    const int64_t rb = static_cast<int64_t>(b) * N, pb = static_cast<int64_t>(b) * (N + 1);
+    // thread tid owns sorted positions [p0, p1); its sums, then an exclusive scan over threads
+    const int per = (N + THREADS - 1) / THREADS;
+    const int p0 = min(N, tid * per), p1 = min(N, p0 + per);
+    double a0 = 0.0, a1 = 0.0, a2 = 0.0;
+    for (int p = p0; p < p1; ++p) {
+        const double x = SortKey<T>::value(ka[p]), wt = w ? w[rb + ia[p]] : 1.0;
+        a0 += wt;
+        a1 += wt * x;
+        a2 += wt * x * x;
+    }
+    double i0 = a0, i1 = a1, i2 = a2;   // inclusive scan within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double u0 = __shfl_up_sync(0xffffffffu, i0, o);
+        const double u1 = __shfl_up_sync(0xffffffffu, i1, o);
+        const double u2 = __shfl_up_sync(0xffffffffu, i2, o);
+        if (lane >= o) {
+            i0 += u0;
+            i1 += u1;
+            i2 += u2;
+        }
+    }
+    if (lane == 31) {
+        wtot[0][warp] = i0;
+        wtot[1][warp] = i1;
+        wtot[2][warp] = i2;
+    }
+    __syncthreads();
+    double r0 = i0 - a0, r1 = i1 - a1, r2 = i2 - a2;   // exclusive within the warp
+    for (int v = 0; v < warp; ++v) {
+        r0 += wtot[0][v];
+        r1 += wtot[1][v];
+        r2 += wtot[2][v];
+    }
+    if (tid == 0) {
+        P0[pb] = 0.0;
+        P1[pb] = 0.0;
+        P2[pb] = 0.0;
+    }
+    for (int p = p0; p < p1; ++p) {
+        const double x = SortKey<T>::value(ka[p]), wt = w ? w[rb + ia[p]] : 1.0;
+        r0 += wt;
+        r1 += wt * x;
+        r2 += wt * x * x;
+        P0[pb + p + 1] = r0;
+        P1[pb + p + 1] = r1;
+        P2[pb + p + 1] = r2;
+    }
+    for (int p = tid; p < N; p += THREADS) {
+        xs_out[rb + p] = SortKey<T>::value(ka[p]);
+        is_out[rb + p] = ia[p];
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(ITER_WARPS * 32)
+    fit1d_iter_kernel(const float *__restrict__ xs, const int32_t *__restrict__ is,
+                      const double *__restrict__ P0, const double *__restrict__ P1,
+                      const double *__restrict__ P2, int B, int N, int K, int iters,
+                      float *__restrict__ C, int32_t *__restrict__ ids,
+                      double *__restrict__ inertia_hist, float *__restrict__ C_hist) {
+    constexpr unsigned FULL = 0xffffffffu;
+    __shared__ float cx_s[ITER_WARPS][ITER_KMAX];   // rounded centroids, by index
+    __shared__ int rank_s[ITER_WARPS][ITER_KMAX];   // rank of centroid k in (cx, k) order
+    __shared__ int order_s[ITER_WARPS][ITER_KMAX];  // centroid at each rank
+    __shared__ int E_s[ITER_WARPS][ITER_KMAX];      // #points whose nearest centroid has rank <= q
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.x * ITER_WARPS + warp;
+    if (b >= B) return;   // whole warps only; nothing below synchronises the block
+    float *cxw = cx_s[warp];
+    int *rankw = rank_s[warp], *orderw = order_s[warp], *Ew = E_s[warp];
+    const int64_t rb = static_cast<int64_t>(b) * N, pb = static_cast<int64_t>(b) * (N + 1);
+    const float *xr = xs + rb;
+    const bool own = lane < K;   // lane k holds centroid k
+    float cm = own ? C[static_cast<int64_t>(b) * K + lane] : 0.f;
+    if (own && C_hist) C_hist[static_cast<int64_t>(b) * K + lane] = cm;
+    int steps = 0;   // halvings that take a range of N + 1 candidates down to one
+    while ((1 << steps) <= N) ++steps;
+
+    for (int t = 0; t <= iters; ++t) {
+        const bool final_pass = (t == iters);
+        if (final_pass && !ids) break;
+        const float cxk = own ? round_through<T>(cm) : 0.f;
+        if (own) cxw[lane] = cxk;
+        __syncwarp();
+        int r = 0;
+        if (own) {
+            for (int j = 0; j < K; ++j) {
+                const float u = cxw[j];
+                r += (u < cxk) || (u == cxk && j < lane);
+            }
+            rankw[lane] = r;
+            orderw[r] = lane;
+        }
+        __syncwarp();
+        // boundary q = lane: first sorted position whose nearest centroid ranks above q
+        int lo = 0, len = N;
+        for (int st = 0; st < steps; ++st) {
+            const int half = len >> 1;
+            const int mid = lo + half;
+            const float x = len > 0 ? xr[mid] : 0.f;
+            float best = INFINITY;
+            int bi = 0;
+            for (int k = 0; k < K; ++k) {
+                const float dx = x - cxw[k];
+                const float dd = dx * dx;
+                if (dd < best) {
+                    best = dd;
+                    bi = k;
+                }
+            }
+            if (len > 0) {
+                if (rankw[bi] <= lane) {
+                    lo = mid + 1;
+                    len -= half + 1;
+                } else {
+                    len = half;
+                }
+            }
+        }
+        const int Eq = lane < K - 1 ? lo : N;
+        if (own) Ew[lane] = Eq;
+        __syncwarp();
+        if (final_pass) {
+            for (int p = lane; p < N; p += 32) {
+                int q = 0;
+                while (Ew[q] <= p) ++q;
+                ids[rb + is[rb + p]] = orderw[q];
+            }
+            break;
+        }
+        // cluster of rank q = lane: sorted positions [s, Eq), centroid orderw[q]
+        const int s = (own && lane > 0) ? Ew[lane - 1] : 0;
+        double W = 0.0, S = 0.0, Q = 0.0;
+        int cnt = 0;
+        if (own) {
+            cnt = Eq - s;
+            W = P0[pb + Eq] - P0[pb + s];
+            S = P1[pb + Eq] - P1[pb + s];
+            Q = P2[pb + Eq] - P2[pb + s];
+        }
+        const double c = own ? static_cast<double>(cxw[orderw[lane]]) : 0.0;
+        double iner = own ? (Q - 2.0 * c * S) + c * c * W : 0.0;
+        iner = warp_sum(iner);
+        if (lane == 0 && inertia_hist) inertia_hist[static_cast<int64_t>(t) * B + b] = iner;
+        const bool moved = own && cnt > 0 && W > 0.0;
+        const float nv = moved ? __double2float_rn(__ddiv_rn(S, W)) : 0.f;
+        const unsigned moved_mask = __ballot_sync(FULL, moved);
+        const int my_rank = own ? rankw[lane] : 0;
+        const float got = __shfl_sync(FULL, nv, my_rank);
+        if (own && ((moved_mask >> my_rank) & 1u)) cm = got;
+        if (own && C_hist) C_hist[(static_cast<int64_t>(t + 1) * B + b) * K + lane] = cm;
+        __syncwarp();
+    }
+    if (own) C[static_cast<int64_t>(b) * K + lane] = cm;
 }
 
 }  // namespace fit1d

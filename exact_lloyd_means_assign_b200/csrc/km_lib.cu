@@ -86,6 +86,30 @@ inline UpdateWs carve_update(Carver &c, int64_t B, int64_t N, int64_t K, int64_t
     return u;
 }
 
+inline bool fit1d_ok(int64_t N, int64_t K, int64_t d) {
+    return d == 1 && K <= km::fit1d::KMAX && N <= km::fit1d::NMAX;
+}
+// the warp-per-row form: one centroid per lane
+inline bool fit1d_rows_ok(int64_t N, int64_t K, int64_t d) {
+    return fit1d_ok(N, K, d) && K <= km::fit1d::ITER_KMAX;
+}
+
+// Warp-per-row 1-D fit: sorted values and original indices, prefix sums of w, w*x, w*x^2.
+struct Fit1dWs {
+    float *xs;
+    int32_t *is;
+    double *P0, *P1, *P2;
+};
+inline Fit1dWs carve_fit1d(Carver &c, int64_t B, int64_t N) {
+    Fit1dWs g;
+    g.xs = c.take<float>(static_cast<size_t>(B * N) * 4);
+    g.is = c.take<int32_t>(static_cast<size_t>(B * N) * 4);
+    g.P0 = c.take<double>(static_cast<size_t>(B * (N + 1)) * 8);
+    g.P1 = c.take<double>(static_cast<size_t>(B * (N + 1)) * 8);
+    g.P2 = c.take<double>(static_cast<size_t>(B * (N + 1)) * 8);
+    return g;
+}
+
 struct FitWs {
     void *Cx;
     float *cn;
@@ -103,7 +127,9 @@ inline FitWs carve_fit(Carver &c, int64_t B, int64_t N, int64_t K, int64_t d, km
     f.rest = c.base ? c.base + c.off : nullptr;
     Carver u(nullptr);
     carve_update(u, B, N, K, d);
-    c.off += std::max(u.off, ws_assign(B, K, d, dt));
+    Carver g(nullptr);
+    if (fit1d_rows_ok(N, K, d)) carve_fit1d(g, B, N);
+    c.off += std::max({u.off, ws_assign(B, K, d, dt), g.off});
     return f;
 }
 
@@ -582,9 +608,27 @@ km_status do_update_partial(const void *X, km_dtype dt, const int32_t *ids, cons
 
 template <typename T>
 km_status run_fit1d(const void *X, const float *w, int64_t B, int64_t N, int64_t K, float *C,
-                    int iters, int32_t *ids, double *inertia_hist, float *C_hist, cudaStream_t st) {
+                    int iters, int32_t *ids, double *inertia_hist, float *C_hist, void *ws,
+                    cudaStream_t st) {
     int NP = 2;
     while (NP < N) NP <<= 1;
+    if (fit1d_rows_ok(N, K, 1)) {
+        using namespace km::fit1d;
+        Carver r(ws);
+        const Fit1dWs g = carve_fit1d(r, B, N);
+        // the radix sort splits the row into RADIX_WARPS segments of whole 32-position rounds
+        const int NR = static_cast<int>(ceil_div(N, RADIX_WARPS * 32) * RADIX_WARPS * 32);
+        if (cudaFuncSetAttribute(fit1d_sort_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 NMAX * 12) != cudaSuccess)
+            return KM_ERR_CUDA;
+        fit1d_sort_kernel<T><<<static_cast<unsigned>(B), THREADS, static_cast<size_t>(NR) * 12, st>>>(
+            static_cast<const T *>(X), w, static_cast<int>(N), NR, g.xs, g.is, g.P0, g.P1, g.P2);
+        if (launch_status() != KM_OK) return KM_ERR_CUDA;
+        fit1d_iter_kernel<T><<<static_cast<unsigned>(ceil_div(B, ITER_WARPS)), ITER_WARPS * 32, 0, st>>>(
+            g.xs, g.is, g.P0, g.P1, g.P2, static_cast<int>(B), static_cast<int>(N), static_cast<int>(K),
+            iters, C, ids, inertia_hist, C_hist);
+        return launch_status();
+    }
     const size_t smem = static_cast<size_t>(NP) * 12;
     if (cudaFuncSetAttribute(km::fit1d::fit1d_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              km::fit1d::NMAX * 12) != cudaSuccess)
@@ -595,23 +639,19 @@ km_status run_fit1d(const void *X, const float *w, int64_t B, int64_t N, int64_t
     return launch_status();
 }
 
-inline bool fit1d_ok(int64_t N, int64_t K, int64_t d) {
-    return d == 1 && K <= km::fit1d::KMAX && N <= km::fit1d::NMAX;
-}
-
 km_status do_fit(const void *X, km_dtype dt, const float *w, int64_t B, int64_t N, int64_t K,
                  int64_t d, float *C, int iters, int32_t *ids, double *inertia_hist, float *C_hist,
                  void *ws, cudaStream_t st) {
-    if (fit1d_ok(N, K, d)) {
-        switch (dt) {
-            case KM_F32: return run_fit1d<float>(X, w, B, N, K, C, iters, ids, inertia_hist, C_hist, st);
-            case KM_F16: return run_fit1d<__half>(X, w, B, N, K, C, iters, ids, inertia_hist, C_hist, st);
-            default:
-                return run_fit1d<__nv_bfloat16>(X, w, B, N, K, C, iters, ids, inertia_hist, C_hist, st);
-        }
-    }
     Carver c(ws);
     FitWs f = carve_fit(c, B, N, K, d, dt);
+    if (fit1d_ok(N, K, d)) {
+        switch (dt) {
+            case KM_F32: return run_fit1d<float>(X, w, B, N, K, C, iters, ids, inertia_hist, C_hist, f.rest, st);
+            case KM_F16: return run_fit1d<__half>(X, w, B, N, K, C, iters, ids, inertia_hist, C_hist, f.rest, st);
+            default:
+                return run_fit1d<__nv_bfloat16>(X, w, B, N, K, C, iters, ids, inertia_hist, C_hist, f.rest, st);
+        }
+    }
     Carver r(f.rest);
     UpdateWs u = carve_update(r, B, N, K, d);
     void *caug = f.rest;  // assignment scratch shares the update region (used one after the other)
@@ -852,7 +892,7 @@ km_status km_fit(const void *X, km_dtype dtype, const float *w, int64_t B, int64
         (ids && !aligned(ids, 4)) || (inertia_hist && !aligned(inertia_hist, 8)) ||
         (C_hist && !aligned(C_hist, 4)))
         return KM_ERR_INVALID_ARG;
-    if (!fit1d_ok(N, K, d)) {
+    if (!fit1d_ok(N, K, d) || fit1d_rows_ok(N, K, d)) {   // the fused per-row kernel needs none
         Carver c(nullptr);
         carve_fit(c, B, N, K, d, dtype);
         if (!ws || ws_bytes < c.off || !aligned(ws, kAlign)) return KM_ERR_WORKSPACE;

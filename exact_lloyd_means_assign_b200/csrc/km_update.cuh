@@ -311,9 +311,9 @@ __global__ void __launch_bounds__(SEG_THREADS, SEG_BLOCKS_PER_SM)
 // cluster of a row, the end of a run and the flush are warp-uniform (one vector atomic per lane
 // per run). Each warp walks chunks of 32 sorted positions; the chunk's point indices are
 // fetched one chunk ahead, and its rows are loaded R at a time into registers (R rows of
-// V * sizeof(T) bytes per lane = 4 KB per warp) before any of them is summed. With few
-// registers per thread many warps fit on an SM, which is what keeps enough bytes in flight
-// for random row gathers to run at HBM speed.
+// V * sizeof(T) bytes per lane = 2 KB per warp) before any of them is summed. R is what fits
+// in the 64 registers that four blocks per SM allow without spilling: 4 KB per warp spilled
+// and measured 9-17 % slower, fewer warps per SM (more registers) slower still.
 constexpr int ROWS_THREADS = 256;
 constexpr int ROWS_BLOCKS_PER_SM = 4;
 
@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(ROWS_THREADS, ROWS_BLOCKS_PER_SM)
                           float *__restrict__ sums, float *__restrict__ wsum) {
     constexpr unsigned FULL = 0xffffffffu;
     constexpr int d = 32 * V;
-    constexpr int R = 128 / static_cast<int>(V * sizeof(T));   // rows in flight per lane
+    constexpr int R = 64 / static_cast<int>(V * sizeof(T));    // rows in flight per lane
     const int lane = threadIdx.x & 31;
     const int64_t gw = static_cast<int64_t>(blockIdx.x) * (ROWS_THREADS / 32) + (threadIdx.x >> 5);
     if (gw >= static_cast<int64_t>(B) * ranges_per_batch) return;

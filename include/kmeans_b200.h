@@ -164,9 +164,12 @@ km_status km_init_grid1d(const void *X, km_dtype dtype, int64_t B, int64_t N, in
  *   inertia_hist[iters,B] fp64 out or NULL: inertia of iteration t's assignment;
  *   C_hist[iters+1,B,K,d] fp32 out or NULL: the centroids entering each iteration and the final
  *   ones (C_hist[0] = the input C).
- * d == 1 with K <= 64 and N <= 8192 runs one fused kernel per row that keeps the row and its
- * weights on chip for all iterations (the per-row codebook setting of the LeanQuant issue);
- * everything else chains km_prep / km_assign / km_update on the stream.
+ * d == 1 with N <= 8192 (the per-row codebook setting of the LeanQuant issue): for K <= 32 one
+ * kernel sorts every row once and stores the sorted values, indices and fp64 prefix sums of w,
+ * w*x, w*x^2 in the workspace (32 bytes per point), then one kernel runs all iterations with a
+ * warp per row; for 32 < K <= 64 one fused kernel per row keeps the row on chip (no workspace
+ * needed). Everything else chains km_prep / km_assign / km_update on the stream. `ws` must hold
+ * km_workspace_size(KM_OP_FIT, ...) bytes (else KM_ERR_WORKSPACE).
  */
 km_status km_fit(const void *X, km_dtype dtype, const float *w, int64_t B, int64_t N, int64_t K,
                  int64_t d, float *C, int iters, int32_t *ids, double *inertia_hist,
