@@ -349,6 +349,13 @@ def _timed(fn, steps, stream):
     return t0.elapsed_time(t1) / steps
 
 
+def _steps_for(fn, steps, stream, min_s=0.5):
+    """At least ``steps``, and enough for ``min_s`` seconds so that the clock sampler (100 ms
+    period) sees the timed region."""
+    t = _timed(fn, 2, stream)
+    return max(steps, int(min_s * 1e3 / max(t, 1e-3)) + 1)
+
+
 def run_workload(args):
     """The other synthetic workloads of the measurement table, one JSON line each, 1 GPU:
     tiny_exact (latency, fp32 exact path, eager and CUDA-graph replay of a 20-iteration fit),
@@ -381,15 +388,16 @@ def run_workload(args):
 
         for _ in range(args.warmup):
             fit()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fit()
+        steps = _steps_for(g.replay, args.steps, stream)
         with ClockSampler(0) as clk:
-            eager = _timed(fit, args.steps, stream)
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                fit()
-            graph = _timed(g.replay, args.steps, stream)
+            eager = _timed(fit, steps, stream)
+            graph = _timed(g.replay, steps, stream)
         lines.append(dict(base, metric="exact fp32 Lloyd us/iteration (CUDA-core path)",
                           value=graph * 1e3 / iters, unit="us/iter", higher_is_better=False,
-                          ms_per_step=graph,
+                          ms_per_step=graph, steps=steps,
                           eager_us_per_iter=eager * 1e3 / iters,
                           config={"workload": wl.name, "B": Bw, "N": Nw, "K": Kw, "d": Dw,
                                   "iterations_per_step": iters, "launch": "CUDA graph of one km_fit call"},
@@ -409,15 +417,16 @@ def run_workload(args):
 
             for _ in range(args.warmup):
                 fit()
+            steps = _steps_for(fit, args.steps, stream)
             with ClockSampler(0) as clk:
-                ms = _timed(fit, args.steps, stream)
+                ms = _timed(fit, steps, stream)
             clocks = clk.summary()
             # peak: 128 fp32 lanes per SM per clock x SMs x the median SM clock under load
             mhz = clocks.get("sm_mhz") or 1965.0
             alu_peak = 128 * torch.cuda.get_device_properties(dev).multi_processor_count * mhz * 1e6 / 1e12
             ops = 3.0 * Bw * Nw * Kw * iters   # brute-force equivalent: sub, mul, min per pair
             lines.append(dict(base, metric="weighted 1-D per-row fit iter/s (all rows)",
-                              value=iters * 1e3 / ms, unit="iter/s", ms_per_step=ms,
+                              value=iters * 1e3 / ms, unit="iter/s", ms_per_step=ms, steps=steps,
                               config={"workload": wl.name, "B": Bw, "N": Nw, "K": Kw, "d": 1,
                                       "iterations_per_step": iters, "weighted": True, "init": "grid"},
                               roofline={"bound": "alu", "achieved": ops / (ms * 1e-3) / 1e12,

@@ -234,8 +234,8 @@ __global__ void __launch_bounds__(THREADS)
 // with thousands of rows it is latency-bound. Here the per-row state that an iteration needs is
 // reduced once, up front, to arrays in device memory:
 //   fit1d_sort_kernel  (one CTA per row): the sorted values, their original indices and the
-//                      prefix sums P0 = sum w, P1 = sum w*x, P2 = sum w*x^2 over the sorted order
-//                      (fp64, P[0] = 0);
+//                      prefix sums P0 = sum w, P1 = sum w*x and, when the objective is wanted,
+//                      P2 = sum w*x^2 over the sorted order (fp64, P[0] = 0);
 //   fit1d_iter_kernel  (one warp per row, every row resident at once): per iteration the K - 1
 //                      cluster boundaries by binary search over the sorted values (the same
 //                      exact-argmin test as above), then each cluster's weight, weighted sum and
@@ -251,6 +251,7 @@ constexpr int ITER_KMAX = 32;   // one centroid per lane
 template <typename T> struct SortKey;
 template <> struct SortKey<float> {
     static constexpr int BITS = 32;
+    using Word = uint32_t;   // shared-memory key storage
     static __device__ __forceinline__ uint32_t key(float v) {
         const uint32_t u = __float_as_uint(v);
         return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
@@ -261,6 +262,7 @@ template <> struct SortKey<float> {
 };
 template <typename H, int DUMMY> struct SortKey16 {
     static constexpr int BITS = 16;
+    using Word = uint16_t;
     static __device__ __forceinline__ uint32_t key(uint32_t u) {
         return (u & 0x8000u) ? (~u & 0xffffu) : (u | 0x8000u);
     }
@@ -291,8 +293,8 @@ template <> struct SortKey<__nv_bfloat16> : SortKey16<__nv_bfloat16, 0> {
 constexpr int RADIX_WARPS = THREADS / 32;
 constexpr int RADIX_MAX_ROUNDS = NMAX / RADIX_WARPS / 32;
 
-template <int BITS>
-__device__ __forceinline__ void radix_sort_row(uint32_t *ka, uint16_t *ia, uint32_t *kb, uint16_t *ib,
+template <int BITS, typename Word>
+__device__ __forceinline__ void radix_sort_row(Word *ka, uint16_t *ia, Word *kb, uint16_t *ib,
                                                int (*hist)[256], int seg) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int rounds = seg >> 5;
@@ -341,14 +343,14 @@ __device__ __forceinline__ void radix_sort_row(uint32_t *ka, uint16_t *ia, uint3
         for (int r = 0; r < RADIX_MAX_ROUNDS; ++r) {
             if (r < rounds) {
                 const int pos = warp * seg + r * 32 + lane;
-                const uint32_t k = ka[pos];
+                const Word k = ka[pos];
                 const int dst = hist[warp][(k >> shift) & 255] + local[r];
                 kb[dst] = k;
                 ib[dst] = ia[pos];
             }
         }
         __syncthreads();
-        uint32_t *tk = ka;
+        Word *tk = ka;
         ka = kb;
         kb = tk;
         uint16_t *ti = ia;
@@ -358,75 +360,100 @@ __device__ __forceinline__ void radix_sort_row(uint32_t *ka, uint16_t *ia, uint3
 }
 
 template <typename T>
-__global__ void __launch_bounds__(THREADS)
+__global__ void __launch_bounds__(THREADS, 4)
     fit1d_sort_kernel(const T *__restrict__ X, const float *__restrict__ w, int N, int NP,
                       float *__restrict__ xs_out, int32_t *__restrict__ is_out,
                       double *__restrict__ P0, double *__restrict__ P1, double *__restrict__ P2) {
-    // shared memory: two key buffers (uint32) and two index buffers (uint16) of NP = 8 * seg
+    // shared memory: (keys, indices) twice, NP = 8 * seg entries each; keys are 16- or 32-bit
+    // words. The second pair is contiguous, so after the sort it serves as NP floats.
+    using Word = typename SortKey<T>::Word;
     extern __shared__ uint8_t sm[];
-    uint32_t *ka = reinterpret_cast<uint32_t *>(sm);
-    uint32_t *kb = ka + NP;
-    uint16_t *ia = reinterpret_cast<uint16_t *>(kb + NP);
-    uint16_t *ib = ia + NP;
+    Word *ka = reinterpret_cast<Word *>(sm);
+    uint16_t *ia = reinterpret_cast<uint16_t *>(ka + NP);
+    Word *kb = reinterpret_cast<Word *>(ia + NP);
+    uint16_t *ib = reinterpret_cast<uint16_t *>(kb + NP);
     __shared__ int hist[RADIX_WARPS][256];
     __shared__ double wtot[3][THREADS / 32];
     const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const T *xb = X + static_cast<int64_t>(b) * N;
     for (int p = tid; p < NP; p += THREADS) {
-        ka[p] = p < N ? SortKey<T>::key(xb[p]) : 0xffffffffu;
+        ka[p] = static_cast<Word>(p < N ? SortKey<T>::key(xb[p]) : 0xffffffffu);
         ia[p] = static_cast<uint16_t>(p);
     }
     __syncthreads();
-    radix_sort_row<SortKey<T>::BITS>(ka, ia, kb, ib, hist, NP / RADIX_WARPS);
+    radix_sort_row<SortKey<T>::BITS, Word>(ka, ia, kb, ib, hist, NP / RADIX_WARPS);
     // an even number of passes leaves the result in (ka, ia)
     const int64_t rb = static_cast<int64_t>(b) * N, pb = static_cast<int64_t>(b) * (N + 1);
-    // thread tid owns sorted positions [p0, p1); its sums, then an exclusive scan over threads
-    const int per = (N + THREADS - 1) / THREADS;
-    const int p0 = min(N, tid * per), p1 = min(N, p0 + per);
-    double a0 = 0.0, a1 = 0.0, a2 = 0.0;
-    for (int p = p0; p < p1; ++p) {
-        const double x = SortKey<T>::value(ka[p]), wt = w ? w[rb + ia[p]] : 1.0;
-        a0 += wt;
-        a1 += wt * x;
-        a2 += wt * x * x;
-    }
-    double i0 = a0, i1 = a1, i2 = a2;   // inclusive scan within the warp
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const double u0 = __shfl_up_sync(0xffffffffu, i0, o);
-        const double u1 = __shfl_up_sync(0xffffffffu, i1, o);
-        const double u2 = __shfl_up_sync(0xffffffffu, i2, o);
-        if (lane >= o) {
-            i0 += u0;
-            i1 += u1;
-            i2 += u2;
-        }
-    }
-    if (lane == 31) {
-        wtot[0][warp] = i0;
-        wtot[1][warp] = i1;
-        wtot[2][warp] = i2;
-    }
-    __syncthreads();
-    double r0 = i0 - a0, r1 = i1 - a1, r2 = i2 - a2;   // exclusive within the warp
-    for (int v = 0; v < warp; ++v) {
-        r0 += wtot[0][v];
-        r1 += wtot[1][v];
-        r2 += wtot[2][v];
-    }
+    // prefix sums over the sorted order, THREADS positions at a time (coalesced stores); the
+    // running totals before each tile are the same in every thread. P2 may be null (no objective).
     if (tid == 0) {
         P0[pb] = 0.0;
         P1[pb] = 0.0;
-        P2[pb] = 0.0;
+        if (P2) P2[pb] = 0.0;
     }
-    for (int p = p0; p < p1; ++p) {
-        const double x = SortKey<T>::value(ka[p]), wt = w ? w[rb + ia[p]] : 1.0;
-        r0 += wt;
-        r1 += wt * x;
-        r2 += wt * x * x;
-        P0[pb + p + 1] = r0;
-        P1[pb + p + 1] = r1;
-        P2[pb + p + 1] = r2;
+    // the weights in sorted order, gathered 8 per thread at a time into the sort's scratch pair
+    // (free now; at least 4 contiguous bytes per position), before the scan needs them
+    float *wsm = reinterpret_cast<float *>(kb);
+    if (w) {
+        for (int q = 0; q < N; q += 8 * THREADS) {
+            float t8[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int p = q + j * THREADS + tid;
+                t8[j] = p < N ? w[rb + ia[p]] : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int p = q + j * THREADS + tid;
+                if (p < N) wsm[p] = t8[j];
+            }
+        }
+        __syncthreads();
+    }
+    double c0 = 0.0, c1 = 0.0, c2 = 0.0;
+    for (int base = 0; base < N; base += THREADS) {
+        const int p = base + tid;
+        double v0 = 0.0, v1 = 0.0, v2 = 0.0;
+        if (p < N) {
+            const double x = SortKey<T>::value(ka[p]), wt = w ? wsm[p] : 1.f;
+            v0 = wt;
+            v1 = wt * x;
+            v2 = v1 * x;
+        }
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {   // inclusive scan within the warp
+            const double u0 = __shfl_up_sync(0xffffffffu, v0, o);
+            const double u1 = __shfl_up_sync(0xffffffffu, v1, o);
+            const double u2 = __shfl_up_sync(0xffffffffu, v2, o);
+            if (lane >= o) {
+                v0 += u0;
+                v1 += u1;
+                v2 += u2;
+            }
+        }
+        if (lane == 31) {
+            wtot[0][warp] = v0;
+            wtot[1][warp] = v1;
+            wtot[2][warp] = v2;
+        }
+        __syncthreads();
+        double o0 = c0, o1 = c1, o2 = c2;
+        for (int v = 0; v < RADIX_WARPS; ++v) {
+            if (v < warp) {
+                o0 += wtot[0][v];
+                o1 += wtot[1][v];
+                o2 += wtot[2][v];
+            }
+            c0 += wtot[0][v];
+            c1 += wtot[1][v];
+            c2 += wtot[2][v];
+        }
+        if (p < N) {
+            P0[pb + p + 1] = o0 + v0;
+            P1[pb + p + 1] = o1 + v1;
+            if (P2) P2[pb + p + 1] = o2 + v2;
+        }
+        __syncthreads();   // wtot is rewritten by the next tile
     }
     for (int p = tid; p < N; p += THREADS) {
         xs_out[rb + p] = SortKey<T>::value(ka[p]);
@@ -519,12 +546,14 @@ __global__ void __launch_bounds__(ITER_WARPS * 32)
             cnt = Eq - s;
             W = P0[pb + Eq] - P0[pb + s];
             S = P1[pb + Eq] - P1[pb + s];
-            Q = P2[pb + Eq] - P2[pb + s];
+            Q = P2 ? P2[pb + Eq] - P2[pb + s] : 0.0;
         }
         const double c = own ? static_cast<double>(cxw[orderw[lane]]) : 0.0;
-        double iner = own ? (Q - 2.0 * c * S) + c * c * W : 0.0;
-        iner = warp_sum(iner);
-        if (lane == 0 && inertia_hist) inertia_hist[static_cast<int64_t>(t) * B + b] = iner;
+        if (inertia_hist) {   // warp-uniform
+            double iner = own ? (Q - 2.0 * c * S) + c * c * W : 0.0;
+            iner = warp_sum(iner);
+            if (lane == 0) inertia_hist[static_cast<int64_t>(t) * B + b] = iner;
+        }
         const bool moved = own && cnt > 0 && W > 0.0;
         const float nv = moved ? __double2float_rn(__ddiv_rn(S, W)) : 0.f;
         const unsigned moved_mask = __ballot_sync(FULL, moved);

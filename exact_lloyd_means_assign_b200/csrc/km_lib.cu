@@ -618,14 +618,16 @@ km_status run_fit1d(const void *X, const float *w, int64_t B, int64_t N, int64_t
         const Fit1dWs g = carve_fit1d(r, B, N);
         // the radix sort splits the row into RADIX_WARPS segments of whole 32-position rounds
         const int NR = static_cast<int>(ceil_div(N, RADIX_WARPS * 32) * RADIX_WARPS * 32);
+        const size_t per = 2 * (sizeof(typename SortKey<T>::Word) + 2);   // key and index, twice
         if (cudaFuncSetAttribute(fit1d_sort_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 NMAX * 12) != cudaSuccess)
+                                 static_cast<int>(NMAX * per)) != cudaSuccess)
             return KM_ERR_CUDA;
-        fit1d_sort_kernel<T><<<static_cast<unsigned>(B), THREADS, static_cast<size_t>(NR) * 12, st>>>(
-            static_cast<const T *>(X), w, static_cast<int>(N), NR, g.xs, g.is, g.P0, g.P1, g.P2);
+        fit1d_sort_kernel<T><<<static_cast<unsigned>(B), THREADS, static_cast<size_t>(NR) * per, st>>>(
+            static_cast<const T *>(X), w, static_cast<int>(N), NR, g.xs, g.is, g.P0, g.P1,
+            inertia_hist ? g.P2 : nullptr);
         if (launch_status() != KM_OK) return KM_ERR_CUDA;
         fit1d_iter_kernel<T><<<static_cast<unsigned>(ceil_div(B, ITER_WARPS)), ITER_WARPS * 32, 0, st>>>(
-            g.xs, g.is, g.P0, g.P1, g.P2, static_cast<int>(B), static_cast<int>(N), static_cast<int>(K),
+            g.xs, g.is, g.P0, g.P1, inertia_hist ? g.P2 : nullptr, static_cast<int>(B), static_cast<int>(N), static_cast<int>(K),
             iters, C, ids, inertia_hist, C_hist);
         return launch_status();
     }
