@@ -201,6 +201,37 @@ def test_fit1d_weighted_rows_per_iteration(K, cuda_device):
     check_assign(X, C, ids)
 
 
+@pytest.mark.parametrize("dt,N,K,weighted", [
+    ("f32", 3000, 32, True),    # warp-per-row form at its largest K; ragged radix segments
+    ("bf16", 1000, 5, False),
+    ("f16", 8192, 1, True),     # the largest row; one cluster
+    ("f16", 700, 48, True),     # K > 32: the fused one-CTA-per-row form
+])
+def test_fit1d_shapes_per_iteration(dt, N, K, weighted, cuda_device):
+    g = torch.Generator().manual_seed(N + K)
+    B = 6
+    X = (torch.randn((B, N, 1), generator=g) * 0.05).to(DT[dt])
+    X[:, : N // 10] = X[:, N // 10: 2 * (N // 10)]          # repeated values (ties in the sort)
+    w = torch.rand((B, N), generator=g) + 0.01 if weighted else None
+    Xd = X.to(cuda_device)
+    wd = None if w is None else w.to(cuda_device)
+    C = km.km_init_grid1d(Xd, K)
+    iters = 6
+    _, ids, ih, ch = km.km_fit(Xd, C, iters, w=wd, want_ids=True, want_inertia=True, want_hist=True)
+    torch.cuda.synchronize()
+    X64 = oracle.as_f64(X)
+    w64 = None if w is None else oracle.as_f64(w)
+    hist = to_np(ch).astype(np.float64)
+    for t in range(iters):
+        ids_t, d1, d2, inertia = oracle.assign(X64, oracle.round_to_dtype(hist[t], DT[dt]), w64)
+        np.testing.assert_allclose(to_np(ih[t]), inertia, rtol=1e-4)
+        C_ref, _, _ = oracle.update(X64, ids_t, hist[t], w64)
+        for b in range(B):
+            err = np.linalg.norm(hist[t + 1][b] - C_ref[b]) / max(np.linalg.norm(C_ref[b]), 1e-30)
+            assert err <= 1e-3, (t, b, err)
+    check_assign(Xd, C, ids, w=wd)
+
+
 def test_fit1d_unweighted_fp32_and_worked_example(cuda_device):
     from conftest import load_golden
     gold = load_golden("worked_example_weight_clustering.txt")
