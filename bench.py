@@ -7,7 +7,7 @@ larger than the 126 MB L2, so no flush is needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
   python bench.py --out-of-core {batched_assign_bound,single_N33M_K16384} --steps 5
-  python bench.py --workload {tiny_exact,rows_weighted_1d,large_k_assign,contention_update}
+  python bench.py --workload {tiny_exact,rows_weighted_1d,large_k_assign,contention_update,emeans}
 
 A step on the GPU = km_assign (tensor-core FlashAssign; the labels, which is all a Lloyd
 iteration needs: the per-point distance and the inertia are optional outputs) + km_update
@@ -493,6 +493,62 @@ def run_workload(args):
         print(json.dumps(l), flush=True)
 
 
+def run_emeans(args):
+    """e-means against Lloyd on one large problem (the page's heavy setting is 10M points with
+    K = 65536; here B=1, N=2^22, K=16384, d=128, fp16, the same kind of mixture): the time of a
+    2-epoch e-means run (mini-batches of 65536 points, alpha0 = 0.3, cosine decay, splitting of
+    dead clusters between epochs) next to the time of one exact Lloyd iteration at the same size.
+    The page reports e-means matching 25 Lloyd iterations' test error in about 2 epochs."""
+    import exact_lloyd_means_assign_b200 as km
+    import synth
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    Ne, Ke, De, batch, epochs, alpha0 = 1 << 22, 16384, 128, 65536, 2, 0.3
+    d = synth.make_workload(4, device=dev, N=Ne, K=Ke)
+    X, C0 = d["X"], d["C0"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(99)
+    split_u = torch.rand((epochs, 1, Ke), generator=g, device=dev)
+    ws_e = torch.empty(km._load().km_emeans_workspace_size(1, Ke, De, km._dt(X.dtype), 0, batch),
+                       dtype=torch.uint8, device=dev)
+    ws_f = km.workspace(km.KM_OP_FIT, 1, Ne, Ke, De, X.dtype, dev)
+    C = C0.clone()
+
+    def em():
+        C.copy_(C0)
+        km.km_emeans_fit(X, C, batch, epochs, alpha0, split_u=split_u, ws=ws_e, stream=stream)
+
+    def lloyd():
+        C.copy_(C0)
+        km.km_fit(X, C, 1, ws=ws_f, stream=stream)
+
+    for _ in range(args.warmup):
+        em()
+        lloyd()
+    with ClockSampler(0) as clk:
+        em_ms = _timed(em, args.steps, stream)
+        ll_ms = _timed(lloyd, args.steps, stream)
+    peak_tf, _, peak_kind = _peaks()
+    flop_epoch = 2.0 * Ne * Ke * De
+    print(json.dumps({
+        "metric": "e-means 2-epoch fit time (vs one Lloyd iteration at the same size)",
+        "value": em_ms / 1e3, "unit": "s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": em_ms, "higher_is_better": False, "scaling": "none", "vs_baseline": None,
+        "dtype": "f16", "data": "synthetic",
+        "config": {"workload": "emeans_large_k: B=1 N=2^22 K=16384 d=128 fp16 (8192-comp GMM)",
+                   "batch": batch, "epochs": epochs, "alpha0": alpha0, "splitting": True},
+        "emeans_ms_per_epoch": em_ms / epochs, "lloyd_ms_per_iteration": ll_ms,
+        "lloyd_25_iterations_s": 25 * ll_ms / 1e3,
+        "roofline": {"bound": "tensor", "achieved": flop_epoch * epochs / (em_ms * 1e-3) / 1e12,
+                     "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": flop_epoch * epochs / (em_ms * 1e-3) / 1e12 / peak_tf,
+                     "note": "assignment contraction of every point once per epoch over the whole run",
+                     "peak_source": f"{peak_kind} bf16 dense"},
+        "clocks": clk.summary(), "device_error": km.km_device_error()}), flush=True)
+
+
 OOC_WORKLOADS = {
     # name: (synth workload, K override, points per batch element per chunk)
     "batched_assign_bound": (3, None, 16384),
@@ -566,13 +622,16 @@ def main():
     ap.add_argument("--out-of-core", choices=sorted(OOC_WORKLOADS), default=None,
                     help="time the streamed fit (points in host memory) instead of the step")
     ap.add_argument("--workload", default=None,
-                    choices=["tiny_exact", "rows_weighted_1d", "large_k_assign", "contention_update"],
+                    choices=["tiny_exact", "rows_weighted_1d", "large_k_assign", "contention_update",
+                             "emeans"],
                     help="time one of the other synthetic workloads instead of the headline one")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.out_of_core:
         run_out_of_core(args)
+    elif args.workload == "emeans":
+        run_emeans(args)
     elif args.workload:
         run_workload(args)
     elif args.impl == "reference":

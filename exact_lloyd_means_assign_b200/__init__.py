@@ -46,7 +46,7 @@ def _load():
             f"{_LIB_PATH} is missing: build it with `python -m exact_lloyd_means_assign_b200.build` "
             "(or __graft_entry__.build()); there is no fallback implementation")
     lib = ctypes.CDLL(_LIB_PATH)
-    P, I64, I, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    P, I64, I, SZ, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
     sig = {
         "km_status_string": ([I], ctypes.c_char_p),
         "km_abi_version": ([], I),
@@ -64,6 +64,9 @@ def _load():
         "km_update_noalloc": ([P, I, P, P, I64, I64, I64, I64, P, P, P, P, P], I),
         "km_noalloc_scratch_needed": ([I64, I64, I64, I64], SZ),
         "km_stream_workspace_size": ([I64, I64, I64, I, I, I64], SZ),
+        "km_emeans_workspace_size": ([I64, I64, I64, I, I, I64], SZ),
+        "km_emeans_fit": ([P, I, P, I64, I64, I64, I64, P, I64, I, F, P, F, P, P, SZ, P], I),
+        "km_split_dead": ([P, P, P, F, I64, I64, I64, P, P, P, P], I),
         "km_fit_stream": ([P, I, P, I64, I64, I64, I64, P, I, I64, P, P, SZ, P], I),
     }
     for name, (args, res) in sig.items():
@@ -286,6 +289,43 @@ def km_fit_stream(X_host, C, iters, chunk, w_host=None, want_inertia=False, ws=N
         _p(X_host), _dt(X_host.dtype), _p(w_host), B, N, K, d, _p(C), iters, chunk, _p(inertia),
         _p(ws), ws.numel(), _s(stream)))
     return C, inertia
+
+
+def km_emeans_fit(X, C, batch, epochs, alpha0, w=None, split_u=None, split_eps=1.0 / 1024,
+                  want_sse=False, ws=None, stream=None):
+    """e-means run on device tensors: X [B,N,d], C [B,K,d] fp32 updated in place; split_u
+    [epochs,B,K] fp32 uniforms or None. Returns (C, sse_hist [epochs,B] fp64 or None)."""
+    B, N, d = X.shape
+    K = C.shape[1]
+    dev = X.device
+    _need(X, "X")
+    _need(C, "C", torch.float32, (B, K, d), dev)
+    _need(w, "w", torch.float32, (B, N), dev)
+    _need(split_u, "split_u", torch.float32, (epochs, B, K), dev)
+    sse = torch.empty((epochs, B), dtype=torch.float64, device=dev) if want_sse and epochs else None
+    if ws is None:
+        n = _load().km_emeans_workspace_size(B, K, d, _dt(X.dtype), int(w is not None), min(batch, N))
+        ws = torch.empty(max(int(n), 1), dtype=torch.uint8, device=dev)
+    _check("km_emeans_fit", _load().km_emeans_fit(
+        _p(X), _dt(X.dtype), _p(w), B, N, K, d, _p(C), batch, epochs, float(alpha0), _p(split_u),
+        float(split_eps), _p(sse), _p(ws), ws.numel(), _s(stream)))
+    return C, sse
+
+
+def km_split_dead(C, sizes, u, eps=1.0 / 1024, Nc=None, S=None, want_donors=False, stream=None):
+    """Revive clusters with sizes == 0 by proportional splitting (in place on C, sizes, Nc, S).
+    C [B,K,d], sizes/u/Nc [B,K], S [B,K,d] fp32 device tensors. Returns donors [B,K] or None."""
+    B, K, d = C.shape
+    dev = C.device
+    _need(C, "C", torch.float32, None, dev)
+    _need(sizes, "sizes", torch.float32, (B, K), dev)
+    _need(u, "u", torch.float32, (B, K), dev)
+    _need(Nc, "Nc", torch.float32, (B, K), dev)
+    _need(S, "S", torch.float32, (B, K, d), dev)
+    donors = torch.empty((B, K), dtype=torch.int32, device=dev) if want_donors else None
+    _check("km_split_dead", _load().km_split_dead(
+        _p(C), _p(sizes), _p(u), float(eps), B, K, d, _p(Nc), _p(S), _p(donors), _s(stream)))
+    return donors
 
 
 def km_assign_uses_tensor_cores(X, Cx):

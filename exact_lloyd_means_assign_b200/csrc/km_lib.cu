@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 
@@ -16,6 +17,7 @@
 #include "km_assign_tc.cuh"
 #include "km_centroids.cuh"
 #include "km_common.cuh"
+#include "km_emeans.cuh"
 #include "km_fit1d.cuh"
 #include "km_update.cuh"
 
@@ -761,6 +763,138 @@ km_status do_fit_stream(const void *Xh, km_dtype dt, const float *wh, int64_t B,
     return s;
 }
 
+// e-means: state, epoch totals, one mini-batch's statistics and one problem's batch scratch.
+struct EmeansWs {
+    void *Cx;
+    float *cn, *S, *Nc, *eS, *eW, *bsum, *bw, *sizes;
+    int32_t *ids, *eCnt, *bcnt;
+    UpdateWs u;
+    void *caug;
+};
+inline EmeansWs carve_emeans(Carver &c, int64_t B, int64_t K, int64_t d, km_dtype dt, int64_t batch) {
+    EmeansWs e;
+    const size_t kd = static_cast<size_t>(B * K * d), bk = static_cast<size_t>(B * K);
+    e.Cx = c.take<uint8_t>(kd * dtype_size(dt));
+    e.cn = c.take<float>(bk * 4);
+    e.S = c.take<float>(kd * 4);
+    e.Nc = c.take<float>(bk * 4);
+    e.eS = c.take<float>(kd * 4);
+    e.eW = c.take<float>(bk * 4);
+    e.bsum = c.take<float>(kd * 4);
+    e.bw = c.take<float>(bk * 4);
+    e.sizes = c.take<float>(bk * 4);
+    e.ids = c.take<int32_t>(static_cast<size_t>(batch) * 4);
+    e.eCnt = c.take<int32_t>(bk * 4);
+    e.bcnt = c.take<int32_t>(bk * 4);
+    e.u = carve_update(c, 1, batch, K, d);
+    e.caug = c.base ? c.base + c.off : nullptr;
+    c.off += align_up(ws_assign(1, K, d, dt));
+    return e;
+}
+
+template <typename T>
+km_status run_ema(const float *s, const int32_t *cnt, const float *wsum, float alpha, int64_t rows,
+                  int64_t d, float *S, float *Nc, float *C, void *Cx, float *cn, float *eS,
+                  int32_t *eCnt, float *eW, cudaStream_t st) {
+    constexpr int WPB = 8;
+    km::em::ema_kernel<T><<<static_cast<unsigned>(ceil_div(rows, WPB)), WPB * 32, 0, st>>>(
+        s, cnt, wsum, alpha, rows, static_cast<int>(d), S, Nc, C, static_cast<T *>(Cx), cn, eS,
+        eCnt, eW);
+    return launch_status();
+}
+
+km_status ema_dispatch(km_dtype dt, const float *s, const int32_t *cnt, const float *wsum,
+                       float alpha, int64_t rows, int64_t d, float *S, float *Nc, float *C,
+                       void *Cx, float *cn, float *eS, int32_t *eCnt, float *eW, cudaStream_t st) {
+    switch (dt) {
+        case KM_F16: return run_ema<__half>(s, cnt, wsum, alpha, rows, d, S, Nc, C, Cx, cn, eS, eCnt, eW, st);
+        case KM_BF16:
+            return run_ema<__nv_bfloat16>(s, cnt, wsum, alpha, rows, d, S, Nc, C, Cx, cn, eS, eCnt, eW, st);
+        default: return run_ema<float>(s, cnt, wsum, alpha, rows, d, S, Nc, C, Cx, cn, eS, eCnt, eW, st);
+    }
+}
+
+km_status run_split(float *sizes, const float *u, float eps, int64_t B, int64_t K, int64_t d,
+                    float *C, float *Nc, float *S, int32_t *donors, cudaStream_t st) {
+    km::em::split_kernel<<<static_cast<unsigned>(B), km::em::SPLIT_THREADS, 0, st>>>(
+        sizes, u, eps, static_cast<int>(K), static_cast<int>(d), C, Nc, S, donors);
+    return launch_status();
+}
+
+// Step size of step t of T: cosine decay from alpha0 towards 0.1 alpha0 (evaluated in fp64).
+inline float emeans_alpha(float alpha0, int64_t t, int64_t T) {
+    const double pi = 3.14159265358979323846;
+    return static_cast<float>(static_cast<double>(alpha0) *
+                              (0.1 + 0.9 * (1.0 + std::cos(pi * static_cast<double>(t) /
+                                                           static_cast<double>(T))) / 2.0));
+}
+
+// The e-means run: consecutive mini-batches of `batch` points per problem, each assigned against
+// the current centroids and folded into the moving averages; dead clusters (no point in an
+// epoch) split between epochs when uniforms are given; at the end the centroids move to the mean
+// of the points the last epoch assigned to them.
+km_status do_emeans(const void *X, km_dtype dt, const float *w, int64_t B, int64_t N, int64_t K,
+                    int64_t d, float *C, int64_t batch, int epochs, float alpha0,
+                    const float *split_u, float eps, double *sse_hist, void *ws, cudaStream_t st) {
+    Carver c(ws);
+    EmeansWs e = carve_emeans(c, B, K, d, dt, batch);
+    const size_t esz = dtype_size(dt);
+    const int64_t rows = B * K;
+    const size_t kd4 = static_cast<size_t>(rows * d) * 4;
+    if (cudaMemcpyAsync(e.S, C, kd4, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return KM_ERR_CUDA;
+    km::em::fill_f32_kernel<<<static_cast<unsigned>(ceil_div(rows, 256)), 256, 0, st>>>(e.Nc, 1.f, rows);
+    if (launch_status() != KM_OK) return KM_ERR_CUDA;
+    km_status s = prep_dispatch(C, dt, rows, d, e.Cx, e.cn, st);
+    if (s != KM_OK) return s;
+    const int64_t steps = ceil_div(N, batch), T = static_cast<int64_t>(epochs) * steps;
+    for (int ep = 0; ep < epochs; ++ep) {
+        double *sse = sse_hist ? sse_hist + static_cast<int64_t>(ep) * B : nullptr;
+        if (cudaMemsetAsync(e.eS, 0, kd4, st) != cudaSuccess ||
+            cudaMemsetAsync(e.eCnt, 0, static_cast<size_t>(rows) * 4, st) != cudaSuccess ||
+            cudaMemsetAsync(e.eW, 0, static_cast<size_t>(rows) * 4, st) != cudaSuccess ||
+            (sse && cudaMemsetAsync(sse, 0, static_cast<size_t>(B) * 8, st) != cudaSuccess))
+            return KM_ERR_CUDA;
+        for (int64_t stp = 0; stp < steps; ++stp) {
+            const int64_t n0 = stp * batch, n = std::min(batch, N - n0);
+            for (int64_t b = 0; b < B; ++b) {
+                const void *Xb = static_cast<const uint8_t *>(X) + static_cast<size_t>((b * N + n0) * d) * esz;
+                const float *wb = w ? w + b * N + n0 : nullptr;
+                const void *Cxb = static_cast<const uint8_t *>(e.Cx) + static_cast<size_t>(b * K * d) * esz;
+                s = do_assign(Xb, dt, Cxb, e.cn + b * K, wb, 1, n, K, d, e.ids, nullptr,
+                              sse ? sse + b : nullptr, e.caug, st, true);
+                if (s != KM_OK) return s;
+                s = do_update_partial(Xb, dt, e.ids, wb, 1, n, K, d, e.bsum + b * K * d,
+                                      w ? e.bw + b * K : nullptr, e.bcnt + b * K, e.u, st);
+                if (s != KM_OK) return s;
+            }
+            s = ema_dispatch(dt, e.bsum, e.bcnt, w ? e.bw : nullptr,
+                             emeans_alpha(alpha0, static_cast<int64_t>(ep) * steps + stp, T), rows, d,
+                             e.S, e.Nc, C, e.Cx, e.cn, e.eS, e.eCnt, w ? e.eW : nullptr, st);
+            if (s != KM_OK) return s;
+        }
+        if (split_u && ep + 1 < epochs) {
+            // sizes = the epoch's point counts (weight sums when weighted)
+            if (w) {
+                if (cudaMemcpyAsync(e.sizes, e.eW, static_cast<size_t>(rows) * 4,
+                                    cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+                    return KM_ERR_CUDA;
+            } else {
+                km::em::i32_to_f32_kernel<<<static_cast<unsigned>(ceil_div(rows, 256)), 256, 0, st>>>(
+                    e.eCnt, e.sizes, rows);
+                if (launch_status() != KM_OK) return KM_ERR_CUDA;
+            }
+            s = run_split(e.sizes, split_u + static_cast<int64_t>(ep) * rows, eps, B, K, d, C, e.Nc,
+                          e.S, nullptr, st);
+            if (s != KM_OK) return s;
+            s = prep_dispatch(C, dt, rows, d, e.Cx, e.cn, st);
+            if (s != KM_OK) return s;
+        }
+    }
+    if (epochs > 0)
+        return finalize_dispatch(e.eS, w ? e.eW : nullptr, e.eCnt, C, rows, d, C, dt, e.Cx, e.cn, st);
+    return KM_OK;
+}
+
 }  // namespace
 
 // =================================================================== exported C ABI
@@ -922,6 +1056,41 @@ km_status km_fit_stream(const void *X_host, km_dtype dtype, const float *w_host,
         !aligned(ws, kAlign))
         return KM_ERR_WORKSPACE;
     return do_fit_stream(X_host, dtype, w_host, B, N, K, d, C, iters, chunk, inertia_hist, ws, S(stream));
+}
+
+size_t km_emeans_workspace_size(int64_t B, int64_t K, int64_t d, km_dtype dtype, int weighted,
+                                int64_t batch) {
+    (void)weighted;   // the weight-sum arrays are always carved
+    if (!sizes_ok(B, batch, K, d) || !valid_dtype(dtype)) return 0;
+    Carver c(nullptr);
+    carve_emeans(c, B, K, d, dtype, batch);
+    return c.off;
+}
+
+km_status km_emeans_fit(const void *X, km_dtype dtype, const float *w, int64_t B, int64_t N,
+                        int64_t K, int64_t d, float *C, int64_t batch, int epochs, float alpha0,
+                        const float *split_u, float split_eps, double *sse_hist, void *ws,
+                        size_t ws_bytes, void *stream) {
+    if (!X || !C || epochs < 0 || !valid_dtype(dtype) || !sizes_ok(B, N, K, d) || batch < 1 ||
+        !(alpha0 > 0.f && alpha0 <= 1.f) || !(split_eps >= 0.f && split_eps < 1.f) ||
+        !elem_aligned(X, dtype) || !aligned(C, 4) || (w && !aligned(w, 4)) ||
+        (split_u && !aligned(split_u, 4)) || (sse_hist && !aligned(sse_hist, 8)))
+        return KM_ERR_INVALID_ARG;
+    batch = std::min(batch, N);
+    if (!ws || ws_bytes < km_emeans_workspace_size(B, K, d, dtype, w != nullptr, batch) ||
+        !aligned(ws, kAlign))
+        return KM_ERR_WORKSPACE;
+    return do_emeans(X, dtype, w, B, N, K, d, C, batch, epochs, alpha0, split_u, split_eps,
+                     sse_hist, ws, S(stream));
+}
+
+km_status km_split_dead(float *C, float *sizes, const float *u, float eps, int64_t B, int64_t K,
+                        int64_t d, float *Nc, float *S_sums, int32_t *donors, void *stream) {
+    if (!C || !sizes || !u || !sizes_ok(B, 1, K, d) || !(eps >= 0.f && eps < 1.f) ||
+        !aligned(C, 4) || !aligned(sizes, 4) || !aligned(u, 4) || (Nc && !aligned(Nc, 4)) ||
+        (S_sums && !aligned(S_sums, 4)) || (donors && !aligned(donors, 4)))
+        return KM_ERR_INVALID_ARG;
+    return run_split(sizes, u, eps, B, K, d, C, Nc, S_sums, donors, S(stream));
 }
 
 km_status km_fit_host(const void *X_host, km_dtype dtype, const float *w_host, int64_t B,

@@ -243,6 +243,54 @@ km_status km_update_noalloc(const void *X, km_dtype dtype, const int32_t *ids, c
 /* Bytes of the static scratch km_update_noalloc needs for these sizes (0 on invalid sizes). */
 size_t km_noalloc_scratch_needed(int64_t B, int64_t N, int64_t K, int64_t d);
 
+/*
+ * e-means: mini-batch k-means with moving averages (steinslab daily "Beating 25 Lloyd
+ * Iterations in 2 Epochs", sections "Breaking 70 Years of Full-Batch Inertia...", "Mini-Batch
+ * Stochastic Noise Escapes Local Optima", "Matching 25 Iterations of Error in Just 2 Epochs" and
+ * "Proportional Splitting Resurrects Thousands of Dead Centers").
+ * Each problem's points are visited `epochs` times in consecutive mini-batches of `batch` points
+ * (in the order given; shuffle beforehand). Every mini-batch is assigned against the current
+ * centroids (the same exact argmin as km_assign), its per-cluster sums s and sizes n (counts, or
+ * weight sums) enter the state
+ *     S <- (1 - a_t) S + a_t s,   N <- (1 - a_t) N + a_t n,   C = S / N (kept where N == 0),
+ * with S = C, N = 1 at the start and a_t = alpha0 (0.1 + 0.9 (1 + cos(pi t / T)) / 2) at step t
+ * of T = epochs * ceil(N_points / batch). Between epochs, when split_u is given, every cluster
+ * that received no point during the epoch is revived as in km_split_dead (sizes = the epoch's
+ * counts or weight sums, uniforms split_u[epoch][B][K]). After the last epoch C moves to the
+ * mean of the points that epoch assigned to each cluster (clusters it left empty keep theirs).
+ *   X[B,N,d] in `dtype`, w[B,N] fp32 or NULL, C[B,K,d] fp32 in/out (device);
+ *   split_u: NULL (no splitting) or [epochs,B,K] fp32 uniforms in [0,1) (device);
+ *   sse_hist: NULL or [epochs,B] fp64 out: per epoch, the sum of w * squared distance of every
+ *   point to the centroid it was assigned to when its mini-batch was processed;
+ *   ws: km_emeans_workspace_size(B, K, d, dtype, weighted, batch) bytes (device, 256-B aligned).
+ * Asynchronous on `stream`. Errors: KM_ERR_INVALID_ARG (null X or C, sizes, batch < 1,
+ * alpha0 outside (0,1], split_eps outside [0,1), misaligned), KM_ERR_WORKSPACE, KM_ERR_CUDA.
+ */
+size_t km_emeans_workspace_size(int64_t B, int64_t K, int64_t d, km_dtype dtype, int weighted,
+                                int64_t batch);
+km_status km_emeans_fit(const void *X, km_dtype dtype, const float *w, int64_t B, int64_t N,
+                        int64_t K, int64_t d, float *C, int64_t batch, int epochs, float alpha0,
+                        const float *split_u, float split_eps, double *sse_hist, void *ws,
+                        size_t ws_bytes, void *stream);
+
+/*
+ * Proportional splitting of dead clusters (steinslab e-means daily, section "Proportional
+ * Splitting Resurrects Thousands of Dead Centers"; usable after a Lloyd update with sizes = the
+ * update's counts). Per problem, the clusters with sizes == 0 are revived in index order: dead
+ * cluster i takes as donor the first cluster j whose running size sum exceeds u[i] * (total
+ * size) (fp64), then per coordinate k (s_k = +1 for even k, -1 for odd k)
+ *     C[i][k] = C[j][k] (1 + eps s_k),   C[j][k] <- C[j][k] (1 - eps s_k),
+ * sizes[i] = sizes[j] / 2, sizes[j] -= sizes[i]; when given, Nc is halved the same way and
+ * S_sums[i], S_sums[j] = C * Nc. Nothing happens when every size is 0.
+ *   C[B,K,d], sizes[B,K], u[B,K] fp32; Nc[B,K], S_sums[B,K,d] fp32 or NULL; donors[B,K] int32
+ *   out or NULL (donor of each revived cluster, -1 elsewhere). All device memory.
+ * Asynchronous on `stream`. One block of 1024 threads per problem; each revival rescans the K
+ * sizes. Errors: KM_ERR_INVALID_ARG (null C/sizes/u, sizes, eps outside [0,1), misaligned),
+ * KM_ERR_CUDA.
+ */
+km_status km_split_dead(float *C, float *sizes, const float *u, float eps, int64_t B, int64_t K,
+                        int64_t d, float *Nc, float *S_sums, int32_t *donors, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

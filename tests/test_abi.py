@@ -75,6 +75,10 @@ def test_workspace_sizes(lib):
     assert 2 * 32 * 4096 * 128 * 2 <= s1 and s2 - s1 >= 2 * 32 * 4096 * 128 * 2
     assert lib.km_stream_workspace_size(32, 1024, 128, 1, 1, 4096) >= s1 + 2 * 32 * 4096 * 4
     assert lib.km_stream_workspace_size(32, 1024, 128, 1, 0, 0) == 0
+    # e-means: state (S, epoch sums, batch sums) is 3 * B*K*d fp32, plus one batch's scratch
+    e1 = lib.km_emeans_workspace_size(1, 65536, 128, 1, 0, 1 << 16)
+    assert e1 >= 3 * 65536 * 128 * 4 + (1 << 16) * 8
+    assert lib.km_emeans_workspace_size(1, 65536, 128, 1, 0, 0) == 0
     for op in range(4):
         assert km.km_workspace_size(op, 3, 1000, 17, 24, f16, True, 5) % 256 == 0
 
@@ -114,6 +118,17 @@ def test_argument_errors_return_before_any_launch(lib):
     assert lib.km_fit_stream(null, 1, null, 1, 10, 4, 8, fake, 3, 4, null, fake, 1 << 30, st) == 1
     assert lib.km_fit_stream(fake, 1, null, 1, 10, 4, 8, fake, 3, 0, null, fake, 1 << 30, st) == 1
     assert lib.km_fit_stream(fake, 1, null, 1, 10, 4, 8, fake, 3, 4, null, fake, 16, st) == 3
+    # km_emeans_fit: batch < 1, alpha0 outside (0, 1], workspace too small
+    f = ctypes.c_float
+    assert lib.km_emeans_fit(fake, 1, null, 1, 10, 4, 8, fake, 0, 2, f(0.5), null, f(0.01), null,
+                             fake, 1 << 30, st) == 1
+    assert lib.km_emeans_fit(fake, 1, null, 1, 10, 4, 8, fake, 5, 2, f(1.5), null, f(0.01), null,
+                             fake, 1 << 30, st) == 1
+    assert lib.km_emeans_fit(fake, 1, null, 1, 10, 4, 8, fake, 5, 2, f(0.5), null, f(0.01), null,
+                             fake, 16, st) == 3
+    # km_split_dead: null sizes, eps outside [0, 1)
+    assert lib.km_split_dead(fake, null, fake, f(0.1), 1, 4, 8, null, null, null, st) == 1
+    assert lib.km_split_dead(fake, fake, fake, f(1.0), 1, 4, 8, null, null, null, st) == 1
     # km_init_grid1d: d is implied 1, K must be >= 1
     assert lib.km_init_grid1d(fake, 1, 1, 10, 0, fake, st) == 1
     # km_prep: nothing to write
