@@ -7,7 +7,8 @@ larger than the 126 MB L2, so no flush is needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
   python bench.py --out-of-core {batched_assign_bound,single_N33M_K16384} --steps 5
-  python bench.py --workload {tiny_exact,rows_weighted_1d,large_k_assign,contention_update,emeans}
+  python bench.py --workload {tiny_exact,rows_weighted_1d,large_k_assign,contention_update,emeans,
+                              codebook1d}
 
 A step on the GPU = km_assign (tensor-core FlashAssign; the labels, which is all a Lloyd
 iteration needs: the per-point distance and the inertia are optional outputs) + km_update
@@ -549,6 +550,65 @@ def run_emeans(args):
         "clocks": clk.summary(), "device_error": km.km_device_error()}), flush=True)
 
 
+def run_codebook1d(args):
+    """Per-row 1-D codebooks on the weighted-rows workload (4096 rows x 4096 fp16 values):
+    k-means++ seeding (K = 16), and encoding every value to its uint8 index against a fitted
+    K = 16 codebook. Encoding is bound by HBM: 2 bytes read + 1 byte written per value."""
+    import exact_lloyd_means_assign_b200 as km
+    import synth
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    d = synth.make_workload(2, device=dev, K=16)
+    X, w = d["X"], d["w"]
+    Bc, Nc = X.shape[0], X.shape[1]
+    Kc = 16
+    C = km.km_init_grid1d(X, Kc)
+    km.km_fit(X, C, 30, w=w)
+    codes = torch.empty((Bc, Nc), dtype=torch.uint8, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(5)
+    u = torch.rand((Bc, Kc), generator=g, device=dev)
+
+    def enc():
+        km.km_encode1d(X, C, codes=codes, stream=stream)
+
+    def pp():
+        km.km_init_kmeanspp1d(X, Kc, u, w=w, stream=stream)
+
+    for _ in range(args.warmup):
+        enc()
+        pp()
+    # one encode is shorter than the host-side cost of a call, so the timed unit is a CUDA graph
+    # of 20 encode launches (the kernels run back to back, as in a pipeline)
+    reps = 20
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(reps):
+            km.km_encode1d(X, C, codes=codes)
+    graph.replay()
+    steps = _steps_for(graph.replay, args.steps, stream)
+    with ClockSampler(0) as clk:
+        enc_ms = _timed(graph.replay, steps, stream) / reps
+        pp_ms = _timed(pp, max(3, args.steps), stream)
+    _, peak_bw, peak_kind = _peaks()
+    nbytes = Bc * Nc * (X.element_size() + 1) + Bc * Kc * 4
+    print(json.dumps({
+        "metric": "1-D codebook encode GB/s (uint8 indices, K=16)", "value": nbytes / enc_ms / 1e6,
+        "unit": "GB/s", "n_gpus": 1, "steps": steps, "warmup": args.warmup, "ms_per_step": enc_ms,
+        "higher_is_better": True, "scaling": "none", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": "rows_weighted_1d: 4096 rows x 4096 fp16, K=16 fitted codebooks",
+                   "l2": "inputs (50 MB) below L2 size; steady-state repeated encode"},
+        "values_per_s": Bc * Nc / (enc_ms * 1e-3), "launches_per_graph": reps,
+        "kmeanspp_ms": pp_ms,
+        "roofline": {"bound": "hbm", "achieved": nbytes / enc_ms / 1e6, "peak": peak_bw, "unit": "GB/s",
+                     "frac": nbytes / enc_ms / 1e6 / peak_bw, "algorithmic_bytes": nbytes,
+                     "peak_source": peak_kind},
+        "clocks": clk.summary(), "device_error": km.km_device_error()}), flush=True)
+
+
 OOC_WORKLOADS = {
     # name: (synth workload, K override, points per batch element per chunk)
     "batched_assign_bound": (3, None, 16384),
@@ -623,7 +683,7 @@ def main():
                     help="time the streamed fit (points in host memory) instead of the step")
     ap.add_argument("--workload", default=None,
                     choices=["tiny_exact", "rows_weighted_1d", "large_k_assign", "contention_update",
-                             "emeans"],
+                             "emeans", "codebook1d"],
                     help="time one of the other synthetic workloads instead of the headline one")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -632,6 +692,8 @@ def main():
         run_out_of_core(args)
     elif args.workload == "emeans":
         run_emeans(args)
+    elif args.workload == "codebook1d":
+        run_codebook1d(args)
     elif args.workload:
         run_workload(args)
     elif args.impl == "reference":

@@ -67,6 +67,8 @@ def _load():
         "km_emeans_workspace_size": ([I64, I64, I64, I, I, I64], SZ),
         "km_emeans_fit": ([P, I, P, I64, I64, I64, I64, P, I64, I, F, P, F, P, P, SZ, P], I),
         "km_split_dead": ([P, P, P, F, I64, I64, I64, P, P, P, P], I),
+        "km_encode1d": ([P, I, I64, I64, P, I64, P, P], I),
+        "km_init_kmeanspp1d": ([P, I, P, I64, I64, I64, P, P, P, P], I),
         "km_fit_stream": ([P, I, P, I64, I64, I64, I64, P, I, I64, P, P, SZ, P], I),
     }
     for name, (args, res) in sig.items():
@@ -326,6 +328,33 @@ def km_split_dead(C, sizes, u, eps=1.0 / 1024, Nc=None, S=None, want_donors=Fals
     _check("km_split_dead", _load().km_split_dead(
         _p(C), _p(sizes), _p(u), float(eps), B, K, d, _p(Nc), _p(S), _p(donors), _s(stream)))
     return donors
+
+
+def km_encode1d(X, C, codes=None, stream=None):
+    """uint8 index of the nearest codebook value: X [B,N] (or [B,N,1]), C [B,K] (or [B,K,1])
+    fp32 with K <= 256. Returns codes [B,N] uint8."""
+    B, N = X.shape[0], X.shape[1]
+    K = C.shape[1]
+    _need(X, "X")
+    _need(C, "C", torch.float32, None, X.device)
+    codes = torch.empty((B, N), dtype=torch.uint8, device=X.device) if codes is None else codes
+    _need(codes, "codes", torch.uint8, (B, N), X.device)
+    _check("km_encode1d", _load().km_encode1d(_p(X), _dt(X.dtype), B, N, _p(C), K, _p(codes), _s(stream)))
+    return codes
+
+
+def km_init_kmeanspp1d(X, K, u, w=None, want_chosen=False, stream=None):
+    """k-means++ seeds per row: X [B,N] (or [B,N,1]), u [B,K] fp32 uniforms, w [B,N] or None.
+    Returns (C [B,K,1] fp32, chosen [B,K] int32 or None)."""
+    B, N = X.shape[0], X.shape[1]
+    _need(X, "X")
+    _need(u, "u", torch.float32, (B, K), X.device)
+    _need(w, "w", torch.float32, (B, N), X.device)
+    C = torch.empty((B, K, 1), dtype=torch.float32, device=X.device)
+    chosen = torch.empty((B, K), dtype=torch.int32, device=X.device) if want_chosen else None
+    _check("km_init_kmeanspp1d", _load().km_init_kmeanspp1d(
+        _p(X), _dt(X.dtype), _p(w), B, N, K, _p(u), _p(C), _p(chosen), _s(stream)))
+    return C, chosen
 
 
 def km_assign_uses_tensor_cores(X, Cx):

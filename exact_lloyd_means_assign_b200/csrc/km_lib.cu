@@ -16,6 +16,7 @@
 #include "km_assign_simt.cuh"
 #include "km_assign_tc.cuh"
 #include "km_centroids.cuh"
+#include "km_codebook1d.cuh"
 #include "km_common.cuh"
 #include "km_emeans.cuh"
 #include "km_fit1d.cuh"
@@ -1091,6 +1092,55 @@ km_status km_split_dead(float *C, float *sizes, const float *u, float eps, int64
         (S_sums && !aligned(S_sums, 4)) || (donors && !aligned(donors, 4)))
         return KM_ERR_INVALID_ARG;
     return run_split(sizes, u, eps, B, K, d, C, Nc, S_sums, donors, S(stream));
+}
+
+km_status km_encode1d(const void *X, km_dtype dtype, int64_t B, int64_t N, const float *C,
+                      int64_t K, uint8_t *codes, void *stream) {
+    using namespace km::cb;
+    if (!X || !C || !codes || !valid_dtype(dtype) || !sizes_ok(B, N, K, 1) || K > ENC_KMAX ||
+        B > kMaxGridY || !elem_aligned(X, dtype) || !aligned(C, 4))
+        return KM_ERR_INVALID_ARG;
+    const dim3 grid(static_cast<unsigned>(ceil_div(N, ENC_THREADS * ENC_VPT)), static_cast<unsigned>(B));
+    cudaStream_t st = S(stream);
+    switch (dtype) {
+        case KM_F32:
+            encode1d_kernel<float><<<grid, ENC_THREADS, 0, st>>>(static_cast<const float *>(X), N, C,
+                                                                 static_cast<int>(K), codes);
+            break;
+        case KM_F16:
+            encode1d_kernel<__half><<<grid, ENC_THREADS, 0, st>>>(static_cast<const __half *>(X), N, C,
+                                                                  static_cast<int>(K), codes);
+            break;
+        default:
+            encode1d_kernel<__nv_bfloat16><<<grid, ENC_THREADS, 0, st>>>(
+                static_cast<const __nv_bfloat16 *>(X), N, C, static_cast<int>(K), codes);
+    }
+    return launch_status();
+}
+
+km_status km_init_kmeanspp1d(const void *X, km_dtype dtype, const float *w, int64_t B, int64_t N,
+                             int64_t K, const float *u, float *C, int32_t *chosen, void *stream) {
+    using namespace km::cb;
+    if (!X || !u || !C || !valid_dtype(dtype) || !sizes_ok(B, N, K, 1) ||
+        !elem_aligned(X, dtype) || (w && !aligned(w, 4)) || !aligned(u, 4) || !aligned(C, 4) ||
+        (chosen && !aligned(chosen, 4)))
+        return KM_ERR_INVALID_ARG;
+    if (N > PP_NMAX) return KM_ERR_UNSUPPORTED;
+    cudaStream_t st = S(stream);
+    const unsigned grid = static_cast<unsigned>(B);
+    const int n = static_cast<int>(N), k = static_cast<int>(K);
+    switch (dtype) {
+        case KM_F32:
+            kmeanspp1d_kernel<float><<<grid, PP_THREADS, 0, st>>>(static_cast<const float *>(X), w, n, k, u, C, chosen);
+            break;
+        case KM_F16:
+            kmeanspp1d_kernel<__half><<<grid, PP_THREADS, 0, st>>>(static_cast<const __half *>(X), w, n, k, u, C, chosen);
+            break;
+        default:
+            kmeanspp1d_kernel<__nv_bfloat16><<<grid, PP_THREADS, 0, st>>>(
+                static_cast<const __nv_bfloat16 *>(X), w, n, k, u, C, chosen);
+    }
+    return launch_status();
 }
 
 km_status km_fit_host(const void *X_host, km_dtype dtype, const float *w_host, int64_t B,

@@ -291,6 +291,32 @@ km_status km_emeans_fit(const void *X, km_dtype dtype, const float *w, int64_t B
 km_status km_split_dead(float *C, float *sizes, const float *u, float eps, int64_t B, int64_t K,
                         int64_t d, float *Nc, float *S_sums, int32_t *donors, void *stream);
 
+/*
+ * 1-D codebook encoding (the weight-clustering proposal reposted on wpnews.pro, "Cache-Aware
+ * Weight Clustering ...": values stored as 8-bit indices of shared cluster values). Each value
+ * X[b,i] becomes the index of its nearest centroid C[b,k] (centroids rounded to `dtype`, fp32
+ * squared distance, lowest index on ties: the same decision as km_assign with d = 1), found by
+ * binary search in the per-row sorted codebook.
+ *   X[B,N] in `dtype`, C[B,K] fp32 (any order), codes[B,N] uint8 out; all device memory.
+ * K <= 256; B <= 65535. Asynchronous on `stream`. Errors: KM_ERR_INVALID_ARG, KM_ERR_CUDA.
+ */
+km_status km_encode1d(const void *X, km_dtype dtype, int64_t B, int64_t N, const float *C,
+                      int64_t K, uint8_t *codes, void *stream);
+
+/*
+ * k-means++ seeding of per-row 1-D codebooks (the LeanQuant issue "1D k-means": rows with more
+ * than 8 clusters are seeded by k-means++). Per row, centre 0 is drawn with probability
+ * proportional to w, every next one proportional to w * (squared distance to the nearest centre
+ * so far), distances and masses in fp64; draw k takes the first point whose running mass exceeds
+ * u[b,k] * (total mass), point 0 when no mass is left.
+ *   X[B,N] in `dtype`, w[B,N] fp32 or NULL (unit weights), u[B,K] fp32 uniforms in [0,1),
+ *   C[B,K] fp32 out (the chosen values), chosen[B,K] int32 out or NULL (their indices).
+ * N <= 8192 (else KM_ERR_UNSUPPORTED). One block per row. Asynchronous on `stream`.
+ * Errors: KM_ERR_INVALID_ARG, KM_ERR_UNSUPPORTED, KM_ERR_CUDA.
+ */
+km_status km_init_kmeanspp1d(const void *X, km_dtype dtype, const float *w, int64_t B, int64_t N,
+                             int64_t K, const float *u, float *C, int32_t *chosen, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -129,6 +129,10 @@ def test_argument_errors_return_before_any_launch(lib):
     # km_split_dead: null sizes, eps outside [0, 1)
     assert lib.km_split_dead(fake, null, fake, f(0.1), 1, 4, 8, null, null, null, st) == 1
     assert lib.km_split_dead(fake, fake, fake, f(1.0), 1, 4, 8, null, null, null, st) == 1
+    # km_encode1d: K above 256; km_init_kmeanspp1d: rows longer than 8192 are not provided
+    assert lib.km_encode1d(fake, 1, 1, 10, fake, 257, fake, st) == 1
+    assert lib.km_init_kmeanspp1d(fake, 1, null, 1, 9000, 4, fake, fake, null, st) == 2
+    assert lib.km_init_kmeanspp1d(fake, 1, null, 1, 100, 4, null, fake, null, st) == 1
     # km_init_grid1d: d is implied 1, K must be >= 1
     assert lib.km_init_grid1d(fake, 1, 1, 10, 0, fake, st) == 1
     # km_prep: nothing to write
