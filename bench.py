@@ -11,9 +11,10 @@ larger than the 126 MB L2, so no flush is needed between steps.
                               codebook1d}
 
 A step on the GPU = km_assign (tensor-core FlashAssign; the labels, which is all a Lloyd
-iteration needs: the per-point distance and the inertia are optional outputs) + km_update
-(histogram, scan, scatter, segmented reduce, finalize) + km_prep (cast of the new centroids for
-the next assignment): exactly one iteration of km_fit's loop without the objective. The
+iteration needs: the per-point distance and the inertia are optional outputs) +
+km_update_partial (histogram, scan, scatter, segmented reduce) + km_finalize (the division, with
+the rounded centroids and their norms for the next assignment written by the same kernel):
+exactly one iteration of km_fit's loop without the objective. The
 assignment with the inertia requested is timed separately and reported as
 "assign_with_inertia_ms". Multi-GPU: one process per GPU (torchrun),
 each rank runs its own B=32 workload (independent problems, no data-path collective, weak
@@ -45,7 +46,7 @@ ASSIGN_FLOP = 2.0 * B * N * K * D                       # <x,c> contraction per 
 # algorithmic bytes of the update: X gathered once + ids read twice + perm written and read
 UPDATE_BYTES = B * N * D * 2 + 4 * B * N * 4 + B * K * D * 4 * 2
 ASSIGN_BYTES = B * N * D * 2 + B * K * D * 2 + B * N * 4
-LAUNCHES_PER_STEP = 8   # caug, assign_tc, hist, scan, scatter, segreduce, finalize, prep
+LAUNCHES_PER_STEP = 7   # caug, assign_tc, hist, scan, scatter, segreduce, finalize (+ rounding)
 
 
 def _peaks():
@@ -155,14 +156,18 @@ def run_gpu(args):
     ws_u = km.workspace(km.KM_OP_UPDATE, B, N, K, D, X.dtype, dev)
     ids = torch.empty((B, N), dtype=torch.int32, device=dev)
     counts = torch.empty((B, K), dtype=torch.int32, device=dev)
+    sums = torch.empty((B, K, D), dtype=torch.float32, device=dev)
     inertia = torch.empty((B,), dtype=torch.float64, device=dev)
     Cx, cn = km.km_prep(C, X.dtype)
     stream = torch.cuda.current_stream()
 
+    def update():
+        km.km_update_partial(X, ids, K, sums=sums, counts=counts, ws=ws_u, stream=stream)
+        km.km_finalize(sums, counts, C, C_new=C, Cx=Cx, cn=cn, stream=stream)
+
     def step():
         km.km_assign(X, Cx, cn, ids=ids, ws=ws_a, stream=stream)
-        km.km_update(X, ids, C, C_new=C, counts=counts, ws=ws_u, stream=stream)
-        km.km_prep(C, X.dtype, Cx=Cx, cn=cn, stream=stream)
+        update()
 
     for _ in range(args.warmup):
         step()
@@ -180,8 +185,7 @@ def run_gpu(args):
             e[0].record(stream)
             km.km_assign(X, Cx, cn, ids=ids, ws=ws_a, stream=stream)
             e[1].record(stream)
-            km.km_update(X, ids, C, C_new=C, counts=counts, ws=ws_u, stream=stream)
-            km.km_prep(C, X.dtype, Cx=Cx, cn=cn, stream=stream)
+            update()
             e[2].record(stream)
         t1.record(stream)
         torch.cuda.synchronize()
@@ -448,14 +452,15 @@ def run_workload(args):
         ws_u = km.workspace(km.KM_OP_UPDATE, Bw, Nw, Kw, Dw, X.dtype, dev)
         ids = torch.empty((Bw, Nw), dtype=torch.int32, device=dev)
         counts = torch.empty((Bw, Kw), dtype=torch.int32, device=dev)
+        sums = torch.empty((Bw, Kw, Dw), dtype=torch.float32, device=dev)
         Cx, cn = km.km_prep(C, X.dtype)
 
         def assign():
             km.km_assign(X, Cx, cn, ids=ids, ws=ws_a, stream=stream)
 
         def update():
-            km.km_update(X, ids, C, C_new=C, counts=counts, ws=ws_u, stream=stream)
-            km.km_prep(C, X.dtype, Cx=Cx, cn=cn, stream=stream)
+            km.km_update_partial(X, ids, Kw, sums=sums, counts=counts, ws=ws_u, stream=stream)
+            km.km_finalize(sums, counts, C, C_new=C, Cx=Cx, cn=cn, stream=stream)
 
         for _ in range(args.warmup):
             assign()
@@ -497,7 +502,8 @@ def run_workload(args):
 def run_emeans(args):
     """e-means against Lloyd on one large problem (the page's heavy setting is 10M points with
     K = 65536; here B=1, N=2^22, K=16384, d=128, fp16, the same kind of mixture): the time of a
-    2-epoch e-means run (mini-batches of 65536 points, alpha0 = 0.3, cosine decay, splitting of
+    2-epoch e-means run (mini-batches of --emeans-batch points, by default four full waves of
+    256-point tiles over 74 SM pairs; alpha0 = 0.3, cosine decay, splitting of
     dead clusters between epochs) next to the time of one exact Lloyd iteration at the same size.
     The page reports e-means matching 25 Lloyd iterations' test error in about 2 epochs."""
     import exact_lloyd_means_assign_b200 as km
@@ -506,7 +512,8 @@ def run_emeans(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
-    Ne, Ke, De, batch, epochs, alpha0 = 1 << 22, 16384, 128, 65536, 2, 0.3
+    Ne, Ke, De, epochs, alpha0 = 1 << 22, 16384, 128, 2, 0.3
+    batch = args.emeans_batch
     d = synth.make_workload(4, device=dev, N=Ne, K=Ke)
     X, C0 = d["X"], d["C0"]
     g = torch.Generator(device=dev)
@@ -681,6 +688,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--out-of-core", choices=sorted(OOC_WORKLOADS), default=None,
                     help="time the streamed fit (points in host memory) instead of the step")
+    ap.add_argument("--emeans-batch", type=int, default=4 * 74 * 256,
+                    help="mini-batch size of the e-means workload")
     ap.add_argument("--workload", default=None,
                     choices=["tiny_exact", "rows_weighted_1d", "large_k_assign", "contention_update",
                              "emeans", "codebook1d"],

@@ -206,15 +206,20 @@ def km_update_partial(X, ids, K, w=None, sums=None, wsum=None, counts=None, ws=N
     return sums, wsum, counts
 
 
-def km_finalize(sums, counts, C_prev, wsum=None, C_new=None, cx_dtype=None, stream=None):
-    """Divide (empty clusters keep C_prev). Returns (C_new, Cx or None, cn or None)."""
+def km_finalize(sums, counts, C_prev, wsum=None, C_new=None, cx_dtype=None, Cx=None, cn=None,
+                stream=None):
+    """Divide (empty clusters keep C_prev); with cx_dtype (or Cx/cn given) also the rounded
+    centroids and their squared norms for the next assignment. Returns (C_new, Cx, cn)."""
     B, K, d = sums.shape
     dev = sums.device
     C_new = torch.empty_like(C_prev) if C_new is None else C_new
-    Cx = cn = None
+    if Cx is not None:
+        cx_dtype = Cx.dtype
     if cx_dtype is not None:
-        Cx = torch.empty((B, K, d), dtype=cx_dtype, device=dev)
-        cn = torch.empty((B, K), dtype=torch.float32, device=dev)
+        Cx = torch.empty((B, K, d), dtype=cx_dtype, device=dev) if Cx is None else Cx
+        cn = torch.empty((B, K), dtype=torch.float32, device=dev) if cn is None else cn
+        _need(Cx, "Cx", cx_dtype, (B, K, d), dev)
+        _need(cn, "cn", torch.float32, (B, K), dev)
     _check("km_finalize", _load().km_finalize(
         _p(sums), _p(wsum), _p(counts), _p(C_prev), B, K, d, _p(C_new),
         _dt(cx_dtype or torch.float32), _p(Cx), _p(cn), _s(stream)))
