@@ -47,6 +47,19 @@ def test_every_declared_symbol_is_exported(lib):
         assert re.search(rf"\bT {n}$", out, flags=re.M), n
 
 
+def test_every_declared_symbol_has_a_typed_binding(lib):
+    # the binding sets argtypes/restype for each entry point it marshals; every one the header
+    # declares must be covered, with as many arguments as the header's parameter list
+    hdr = open(os.path.join(ROOT, "include", "kmeans_b200.h")).read()
+    hdr = re.sub(r"/\*.*?\*/", "", hdr, flags=re.S)
+    for n in _declared_functions():
+        fn = getattr(lib, n)
+        assert fn.argtypes is not None, n
+        m = re.search(rf"\b{n}\s*\(([^)]*)\)", hdr)
+        params = [p for p in m.group(1).split(",") if p.strip() and p.strip() != "void"]
+        assert len(fn.argtypes) == len(params), (n, len(fn.argtypes), len(params))
+
+
 def test_status_strings_and_version(lib):
     assert km.km_abi_version() == 1
     assert km.km_status_string(0) == "KM_OK"
