@@ -1098,24 +1098,32 @@ km_status km_encode1d(const void *X, km_dtype dtype, int64_t B, int64_t N, const
                       int64_t K, uint8_t *codes, void *stream) {
     using namespace km::cb;
     if (!X || !C || !codes || !valid_dtype(dtype) || !sizes_ok(B, N, K, 1) || K > ENC_KMAX ||
-        B > kMaxGridY || !elem_aligned(X, dtype) || !aligned(C, 4))
+        !elem_aligned(X, dtype) || !aligned(C, 4))
         return KM_ERR_INVALID_ARG;
-    const dim3 grid(static_cast<unsigned>(ceil_div(N, ENC_THREADS * ENC_VPT)), static_cast<unsigned>(B));
     cudaStream_t st = S(stream);
-    switch (dtype) {
-        case KM_F32:
-            encode1d_kernel<float><<<grid, ENC_THREADS, 0, st>>>(static_cast<const float *>(X), N, C,
-                                                                 static_cast<int>(K), codes);
-            break;
-        case KM_F16:
-            encode1d_kernel<__half><<<grid, ENC_THREADS, 0, st>>>(static_cast<const __half *>(X), N, C,
-                                                                  static_cast<int>(K), codes);
-            break;
-        default:
-            encode1d_kernel<__nv_bfloat16><<<grid, ENC_THREADS, 0, st>>>(
-                static_cast<const __nv_bfloat16 *>(X), N, C, static_cast<int>(K), codes);
+    const size_t esz = dtype_size(dtype);
+    for (int64_t b0 = 0; b0 < B; b0 += kMaxGridY) {   // rows in slices of the grid's y extent
+        const int64_t nb = std::min<int64_t>(kMaxGridY, B - b0);
+        const dim3 grid(static_cast<unsigned>(ceil_div(N, ENC_THREADS * ENC_VPT)), static_cast<unsigned>(nb));
+        const void *Xs = static_cast<const uint8_t *>(X) + static_cast<size_t>(b0 * N) * esz;
+        const float *Cs = C + b0 * K;
+        uint8_t *out = codes + b0 * N;
+        switch (dtype) {
+            case KM_F32:
+                encode1d_kernel<float><<<grid, ENC_THREADS, 0, st>>>(static_cast<const float *>(Xs), N,
+                                                                     Cs, static_cast<int>(K), out);
+                break;
+            case KM_F16:
+                encode1d_kernel<__half><<<grid, ENC_THREADS, 0, st>>>(static_cast<const __half *>(Xs), N,
+                                                                      Cs, static_cast<int>(K), out);
+                break;
+            default:
+                encode1d_kernel<__nv_bfloat16><<<grid, ENC_THREADS, 0, st>>>(
+                    static_cast<const __nv_bfloat16 *>(Xs), N, Cs, static_cast<int>(K), out);
+        }
+        if (launch_status() != KM_OK) return KM_ERR_CUDA;
     }
-    return launch_status();
+    return KM_OK;
 }
 
 km_status km_init_kmeanspp1d(const void *X, km_dtype dtype, const float *w, int64_t B, int64_t N,

@@ -298,7 +298,7 @@ km_status km_split_dead(float *C, float *sizes, const float *u, float eps, int64
  * squared distance, lowest index on ties: the same decision as km_assign with d = 1), found by
  * binary search in the per-row sorted codebook.
  *   X[B,N] in `dtype`, C[B,K] fp32 (any order), codes[B,N] uint8 out; all device memory.
- * K <= 256; B <= 65535. Asynchronous on `stream`. Errors: KM_ERR_INVALID_ARG, KM_ERR_CUDA.
+ * K <= 256. Asynchronous on `stream`. Errors: KM_ERR_INVALID_ARG, KM_ERR_CUDA.
  */
 km_status km_encode1d(const void *X, km_dtype dtype, int64_t B, int64_t N, const float *C,
                       int64_t K, uint8_t *codes, void *stream);
