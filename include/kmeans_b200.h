@@ -12,13 +12,18 @@
  * "Bottleneck 2"; wispaper blog "2. Sort-Inverse Update"). Per-point sample weights and the
  * uniform-grid initialisation linspace(min, max, K) come from the per-row 1-D codebook fitting
  * of the LeanQuant issue "1D k-means" (kmeans_fit with sample_weight).
+ * Beyond one resident Lloyd iteration: an out-of-core fit that streams X from host memory
+ * (km_fit_stream), e-means mini-batch training with moving averages and the proportional
+ * splitting of dead clusters (km_emeans_fit, km_split_dead; steinslab e-means daily), and 1-D
+ * codebook seeding and encoding (km_init_kmeanspp1d, km_encode1d).
  *
  * Conventions for every entry point:
  *   - Layout: row-major, innermost index last. X[B,N,d], C[B,K,d], w[B,N], ids[B,N],
  *     cn[B,K], counts[B,K]. B independent problems ("batches") share nothing.
- *   - Pointers are DEVICE pointers owned by the caller, except in km_fit_host (host pointers,
- *     see there). The library allocates no memory: scratch comes from the caller's workspace,
- *     sized by km_workspace_size. Nothing is retained between calls.
+ *   - Pointers are DEVICE pointers owned by the caller, except the host buffers of km_fit_host
+ *     and km_fit_stream (see there). The library allocates no device memory: scratch comes from
+ *     the caller's workspace, sized by km_workspace_size (km_stream_workspace_size,
+ *     km_emeans_workspace_size). Nothing is retained between calls.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call only enqueues work
  *     on that stream and returns; KM_OK means "validated and enqueued". km_fit_host is the one
  *     synchronous call.
