@@ -11,9 +11,10 @@
 //     acc[i,k] = -<x_i, c_k> + (||x_i||^2 / 2)~ + ||c_k||^2 / 2  =  d(i,k) / 2 - delta_i
 // The first term is the main reduction (fp16/bf16 operands, the A operand negated through the
 // instruction descriptor). The other two are one extra K=16 step with bf16 operands: the point
-// side carries [x1, x2, 1, 1, 1, 0...] with x1 + x2 ~ ||x||^2 / 2 (delta_i is the rounding of that
-// two-piece split, a constant per row that cannot change the argmin and is added back for the
-// reported distance), the centroid side [1, 1, a, b, c, 0...] with a + b + c = ||c||^2 / 2 to about
+// side carries [x1, x2, 1, 1, 1, 0...] with x1 + x2 ~ (1 + 2^-12) ||x||^2 / 2 (delta_i, minus the
+// raise and the rounding of that two-piece split, is a constant per row that cannot change the
+// argmin and is added back for the reported distance; the raise keeps the accumulator positive),
+// the centroid side [1, 1, a, b, c, 0...] with a + b + c = ||c||^2 / 2 to about
 // 2^-27 relative. Padding centroids carry 1e30 so they never win.
 //
 // Because the accumulator is (half) the distance itself, the epilogue keeps the argmin as a
@@ -451,8 +452,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 const int row = lane + rr * 32;
                 const float half_xn =
                     0.5f * tile_row_sqnorm<T>(sgen + L.x_off + xb * NKC * XCHUNK, NKC, row);
-                const float x1 = __bfloat162float(__float2bfloat16_rn(half_xn));
-                const float x2 = __bfloat162float(__float2bfloat16_rn(half_xn - x1));
+                // The split carries ||x||^2/2 raised by 2^-12 of itself. The accumulator is then
+                // d/2 + (about 2^-13 ||x||^2), positive even for a point on its centroid, since
+                // the two-piece split (2^-18 relative) and the fp32 reduction (below 2^-15
+                // ||x||^2) err by less. Keys of positive floats order ties by index the way the
+                // min expects (lowest index wins); delta takes the raise back out of the
+                // reported distance, and a constant per row cannot change the argmin.
+                const float tgt = fmaf(half_xn, 0x1p-12f, half_xn);
+                const float x1 = __bfloat162float(__float2bfloat16_rn(tgt));
+                const float x2 = __bfloat162float(__float2bfloat16_rn(tgt - x1));
                 dbuf[xb * BM + row] = (half_xn - x1) - x2;
                 // Row of the point-side augmentation in the 32-byte-swizzled layout: the two
                 // 16-byte halves of rows 4..7 of every 8-row group trade places.

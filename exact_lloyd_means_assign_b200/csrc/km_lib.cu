@@ -11,6 +11,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "kmeans_b200.h"
 #include "km_assign_simt.cuh"
@@ -1202,21 +1203,53 @@ km_status km_device_error(void *stream, int *code) {
 // Scratch for km_update_noalloc: one file-scope device array, present on every device that
 // loads the library until the process exits. Host code must not hand the array's name to a
 // kernel (on the host it only names a stand-in); its device address comes from
-// cudaGetSymbolAddress, looked up once per device with that device current.
+// cudaGetSymbolAddress, looked up with the device current once per context (normally once per
+// device).
 static __device__ __align__(256) uint8_t g_km_noalloc_scratch[KM_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+        tried = true;
+    }
+    return fn;
+}
+
+// Device address of the scratch array in the current context. The address belongs to the
+// context the module was loaded in, so it is cached per (device, context) and looked up again
+// when the current context changes (e.g. after cudaDeviceReset). The lookup happens with the
+// device current and allocates nothing; a mutex covers first calls from several host threads.
 void *noalloc_scratch_device_ptr() {
-    static void *cache[64] = {nullptr};
+    static std::mutex mu;
+    static CUcontext ctx_of[64] = {nullptr};
+    static void *addr_of[64] = {nullptr};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!cache[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_km_noalloc_scratch) != cudaSuccess || !p) return nullptr;
-        cache[dev] = p;
+    std::lock_guard<std::mutex> lock(mu);
+    CtxGetCurrentFn get = ctx_get_current_fn();
+    CUcontext ctx = nullptr;
+    // null when the runtime has not yet made its context current on this thread
+    if (get && get(&ctx) == CUDA_SUCCESS && ctx && addr_of[dev] && ctx_of[dev] == ctx)
+        return addr_of[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_km_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+    // the lookup made the device's context current: remember the address for that context
+    ctx = nullptr;
+    if (get && get(&ctx) == CUDA_SUCCESS && ctx) {
+        ctx_of[dev] = ctx;
+        addr_of[dev] = p;
     }
-    return cache[dev];
+    return p;
 }
 
 }  // namespace

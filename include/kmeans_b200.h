@@ -225,19 +225,24 @@ km_status km_device_error(void *stream, int *code);
 /*
  * km_update for callers that cannot allocate device memory: the same computation and outputs
  * as km_update, but the scratch (offsets, cursors, permutation, partial sums) lives in one
- * array of the library itself, KM_NOALLOC_SCRATCH_BYTES (32 MiB) per device, reserved when the
- * library is loaded and held until the process exits. No page text has a counterpart: this is
- * an interface convenience, not part of the method.
+ * array of the library itself, KM_NOALLOC_SCRATCH_BYTES (32 MiB) per device. No page text has a
+ * counterpart: this is an interface convenience, not part of the method.
  * Meant for code that must not call cudaMalloc/cudaFree at that point (the allocation calls
  * can synchronise the device and stall other streams, and some embeddings hand the library no
  * allocator at all), so there is no workspace to pass.
+ *   - The array is reserved when the library's CUDA module is first loaded in a context on a
+ *     device, i.e. at the first call of ANY entry point of this library there (CUDA loads
+ *     modules lazily), and it is held until the context is destroyed (normally process exit).
+ *     Callers that never use km_update_noalloc pay for it too.
  *   - Sizes whose scratch exceeds the array (see km_noalloc_scratch_needed) are rejected with
  *     KM_ERR_WORKSPACE before anything is enqueued.
- *   - The first call on a device looks up the array's device address with
- *     cudaGetSymbolAddress (once per device, on the current device); make that first call
- *     before any stream capture.
- *   - Every call uses the same array: calls that can overlap on the GPU (different streams,
- *     or several host threads) race with each other and must be serialised by the caller.
+ *   - The array's device address is looked up with cudaGetSymbolAddress on the first call in
+ *     each context (normally once per device, with that device current) and cached per context;
+ *     after cudaDeviceReset the next call looks it up again in the new context. Make the first
+ *     call on a device before any stream capture.
+ *   - Every call uses the same array and it keeps the last call's contents (each call clears
+ *     what must start at zero): calls that can overlap on the GPU (different streams, or
+ *     several host threads) race with each other and must be serialised by the caller.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  */
 #define KM_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)

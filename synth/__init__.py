@@ -89,25 +89,31 @@ def _component_draw(n, mix, n_comp, g, device, zipf_s=1.1):
 
 
 def gaussian_mixture(B, N, d, n_comp, sigma, *, mean="normal", lo=-5.0, hi=5.0, mix="equal",
-                     zipf_s=1.1, dtype=torch.float16, device="cpu", seed=0, chunk_rows=1 << 20):
+                     zipf_s=1.1, dtype=torch.float16, device="cpu", seed=0, chunk_rows=1 << 20,
+                     return_labels=False):
     """X[B,N,d] drawn from an isotropic Gaussian mixture (one mixture per batch).
 
-    Rows are generated in chunks so that the fp32 temporaries stay bounded.
+    Rows are generated in chunks so that the fp32 temporaries stay bounded. With
+    ``return_labels`` the component each point was drawn from is returned too (int32 [B,N]):
+    a draw of the generator, not a clustering.
     """
     g = _gen(device, seed)
     X = torch.empty((B, N, d), dtype=dtype, device=device)
+    labels = torch.empty((B, N), dtype=torch.int32, device=device) if return_labels else None
     for b in range(B):
         if mean == "uniform":
             mu = lo + (hi - lo) * torch.rand((n_comp, d), generator=g, device=device)
         else:
             mu = torch.randn((n_comp, d), generator=g, device=device)
         comp = _component_draw(N, mix, n_comp, g, device, zipf_s)
+        if labels is not None:
+            labels[b] = comp.to(torch.int32)
         for s in range(0, N, chunk_rows):
             e = min(N, s + chunk_rows)
             rows = mu[comp[s:e]]
             rows.add_(torch.randn((e - s, d), generator=g, device=device), alpha=sigma)
             X[b, s:e] = rows.to(dtype)
-    return X
+    return (X, labels) if return_labels else X
 
 
 def student_t_rows(B, N, nu=5, scale=0.02, *, dtype=torch.float16, device="cpu", seed=0):
@@ -151,12 +157,14 @@ def pick_init_points(X, K, mode, *, seed=0):
     return C0
 
 
-def make_workload(idx, *, device="cpu", seed=None, B=None, N=None, K=None):
+def make_workload(idx, *, device="cpu", seed=None, B=None, N=None, K=None, labels=False):
     """Build inputs for workload ``idx`` (1..5), optionally shrunk along B and N.
 
     Returns a dict with X, w (or None), C0 (fp32, or None for grid init),
     K, iters and the Workload record. The shrunk variants keep the recipe
     (distribution, d, dtype, K unless overridden) and change only sizes.
+    With ``labels`` (mixture workloads) the dict also holds "labels": the component index
+    each point was drawn from (int32 [B,N]); the same seed gives the same X either way.
     """
     wl = WORKLOADS[idx]
     seed = 1234 + idx if seed is None else seed
@@ -165,6 +173,7 @@ def make_workload(idx, *, device="cpu", seed=None, B=None, N=None, K=None):
     K = wl.K[0] if K is None else K
     ex = wl.extra
     w = None
+    lab = None
     if idx == 2:
         X = student_t_rows(B, N, ex["nu"], ex["scale"], dtype=wl.dtype, device=device, seed=seed)
         w = importance_weights(B, N, device=device, seed=seed + 1)
@@ -172,10 +181,16 @@ def make_workload(idx, *, device="cpu", seed=None, B=None, N=None, K=None):
     else:
         X = gaussian_mixture(B, N, wl.d, ex["n_comp"], ex["sigma"], mean=ex["mean"],
                              lo=ex.get("lo", -5.0), hi=ex.get("hi", 5.0), mix=ex.get("mix", "equal"),
-                             zipf_s=ex.get("zipf_s", 1.1), dtype=wl.dtype, device=device, seed=seed)
+                             zipf_s=ex.get("zipf_s", 1.1), dtype=wl.dtype, device=device, seed=seed,
+                             return_labels=labels)
+        if labels:
+            X, lab = X
         C0 = pick_init_points(X, K, wl.init, seed=seed + 2)
-    return {"X": X, "w": w, "C0": C0, "K": K, "iters": wl.iters, "workload": wl,
-            "B": B, "N": N, "d": wl.d}
+    out = {"X": X, "w": w, "C0": C0, "K": K, "iters": wl.iters, "workload": wl,
+           "B": B, "N": N, "d": wl.d}
+    if labels:
+        out["labels"] = lab
+    return out
 
 
 def describe(idx):

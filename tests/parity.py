@@ -86,6 +86,48 @@ def check_update(X, ids_gpu, C_prev, C_new_gpu, counts_gpu, *, w=None, wsum_gpu=
     return C_ref
 
 
+def oracle_update_chunked(X, ids, C_prev, chunk=1 << 21):
+    """The oracle's update of all of X (on the device) fed the given assignment, chunk by chunk.
+
+    Each chunk's per-cluster means and counts come from ``oracle.update``; the chunk's sums are
+    rebuilt as mean x count (an fp64 rounding, 2^-52 relative) and added in fp64, so the
+    whole-set means are the oracle's own, only regrouped. Returns (C_ref, counts)."""
+    Bx, Nx, dx = X.shape
+    Kx = C_prev.shape[1]
+    C64 = oracle.as_f64(C_prev.cpu())
+    S = np.zeros((Bx, Kx, dx))
+    cnt = np.zeros((Bx, Kx), np.int64)
+    for b in range(Bx):
+        for s in range(0, Nx, chunk):
+            Xc = oracle.as_f64(X[b:b + 1, s:s + chunk].cpu())
+            Cc, nc, _ = oracle.update(Xc, to_np(ids[b:b + 1, s:s + chunk]), C64[b:b + 1])
+            S[b] += Cc[0] * nc[0][:, None]
+            cnt[b] += nc[0]
+    nz = cnt > 0
+    C_ref = C64.copy()
+    C_ref[nz] = S[nz] / cnt[nz][:, None]
+    return C_ref, cnt
+
+
+def oracle_inertia_of(X, ids, C, dtype, chunk=1 << 21):
+    """sum_i ||x_i - c_{ids_i}||^2 per batch element, every distance from the oracle: the
+    points of each cluster are assigned against that one (rounded) centroid."""
+    Bx, Nx, _ = X.shape
+    Cr = oracle.round_to_dtype(C.cpu(), dtype)
+    tot = np.zeros(Bx)
+    for b in range(Bx):
+        for s in range(0, Nx, chunk):
+            Xc = oracle.as_f64(X[b, s:s + chunk].cpu())
+            ic = to_np(ids[b, s:s + chunk])
+            order = np.argsort(ic, kind="stable")
+            ks, starts = np.unique(ic[order], return_index=True)
+            ends = np.append(starts[1:], len(order))
+            for k, a, e in zip(ks, starts, ends):
+                _, _, _, inert = oracle.assign(Xc[order[a:e]][None], Cr[b, k][None, None])
+                tot[b] += inert[0]
+    return tot
+
+
 def mixture(B, N, d, K, dtype, device, seed=0, sigma=0.3, c_noise=0.3):
     """Clustered points plus K initial centroids drawn among them (plus ``c_noise`` noise)."""
     g = torch.Generator(device="cpu")

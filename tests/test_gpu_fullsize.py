@@ -1,9 +1,10 @@
 """Full-size workloads on the GPU, in the launch configuration the benchmark times.
 
-The oracle cannot evaluate B*N*K*d fp64 work at these sizes in seconds, so the assignment is
-checked on sampled points (each one computed exactly by the oracle), the counts are checked for
-every cluster against a host bincount of the GPU's assignment, and centroids are checked for
-sampled clusters (the largest included) against the fp64 mean of their members.
+The oracle cannot evaluate B*N*K*d fp64 assignment work at these sizes in seconds, so the
+assignment is checked on a large seeded sample of points (each one against every centroid, by
+the oracle). The update is checked for every point: the oracle's update fed the GPU's own
+assignment, chunk by chunk for the 8.6 GB workload. The full-size objective is checked against
+the oracle's distance of every point to the centroid the kernel chose.
 """
 import numpy as np
 import pytest
@@ -12,7 +13,7 @@ import torch
 import exact_lloyd_means_assign_b200 as km
 import oracle
 import synth
-from parity import check_assign, to_np
+from parity import check_assign, oracle_inertia_of, oracle_update_chunked, to_np
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -30,26 +31,17 @@ def _sample_rows(B, N, m, seed):
     return torch.randint(0, B, (m,), generator=g), torch.randint(0, N, (m,), generator=g)
 
 
-def _check_centroids(X, ids, C_prev, C_new, counts, clusters, b=0):
-    """Each sampled non-empty cluster's centroid is the fp64 mean of its members."""
-    idb = ids[b]
-    for k in clusters:
-        k = int(k)
-        members = torch.nonzero(idb == k).flatten()
-        assert members.numel() == int(counts[b, k])
-        if members.numel() == 0:
-            assert torch.equal(C_new[b, k], C_prev[b, k])
-            continue
-        s = np.zeros(X.shape[-1], np.float64)
-        for c0 in range(0, members.numel(), 1 << 19):
-            s += X[b, members[c0:c0 + (1 << 19)]].double().sum(0).cpu().numpy()
-        ref = s / members.numel()
-        got = C_new[b, k].double().cpu().numpy()
-        assert np.linalg.norm(got - ref) <= 1e-3 * max(np.linalg.norm(ref), 1e-30), k
+# sampled points per workload for the assignment check (the oracle's time grows with K)
+ASSIGN_SAMPLE = {3: 65536, 4: 65536, 5: 262144}
 
 
 @pytest.mark.parametrize("idx", [3, 4, 5])
-def test_one_full_iteration(idx, cuda_device):
+def test_full_size_iteration_against_oracle(idx, cuda_device):
+    """One Lloyd iteration of a full-size workload in the benchmark's launch configuration:
+    the assignment on a large seeded sample of points (each against every centroid, by the
+    oracle), the update of every point through the oracle (fed the GPU's own assignment: counts
+    exact, centroids within 1e-3 relative per problem and per cluster, empty clusters unchanged),
+    and the full-size objective against the oracle's distances to the assigned centroids."""
     d = synth.make_workload(idx, device=cuda_device)
     X, C = d["X"], d["C0"]
     B, N, dd = X.shape
@@ -59,41 +51,31 @@ def test_one_full_iteration(idx, cuda_device):
     ids, mind, inertia = km.km_assign(X, Cx, cn, want_mind=True, want_inertia=True)
     C_new, counts, _ = km.km_update(X, ids, C)
     torch.cuda.synchronize()
-    # assignment: sampled points, each against the full centroid set, exactly
-    m = 1024 if idx == 5 else 2048
+    # assignment: a seeded sample, each point against the full centroid set, exactly
+    m = ASSIGN_SAMPLE[idx]
     rows = _sample_rows(B, N, m, seed=idx)
     near = check_assign(X, C, ids, mind_gpu=mind, rows=rows)
+    print(f"workload {idx}: {m} sampled points, 0 mismatches outside near-ties, {near} near-ties")
     assert near <= 0.03 * m      # near-ties may differ; they remain a small minority
-    # counts: every cluster, from the GPU's own assignment
-    ids_h = to_np(ids)
-    for b in range(B):
-        np.testing.assert_array_equal(to_np(counts[b]), np.bincount(ids_h[b], minlength=K))
-    assert int(counts.sum()) == B * N
-    # inertia = sum of the reported per-point distances
-    np.testing.assert_allclose(to_np(inertia), to_np(mind.double().sum(1)), rtol=1e-6)
-    # centroids: sampled clusters plus the largest one, per checked batch
-    for b in ([0, B - 1] if B > 1 else [0]):
-        cb = to_np(counts[b])
-        g = np.random.default_rng(idx + b)
-        pick = set(g.choice(K, 24, replace=False).tolist()) | {int(cb.argmax())}
-        if (cb == 0).any():
-            pick.add(int(np.flatnonzero(cb == 0)[0]))
-        _check_centroids(X, ids, C, C_new, counts, sorted(pick), b=b)
-
-
-def test_full_batch_update_against_oracle(cuda_device):
-    """Workload 3 at full N for two batches: the whole update against the oracle."""
-    d = synth.make_workload(3, B=2, device=cuda_device)
-    X, C = d["X"], d["C0"]
-    Cx, cn = km.km_prep(C, X.dtype)
-    ids, _, _ = km.km_assign(X, Cx, cn)
-    C_new, counts, _ = km.km_update(X, ids, C)
-    torch.cuda.synchronize()
-    C_ref, cnt_ref, _ = oracle.update(oracle.as_f64(X.cpu()), to_np(ids), oracle.as_f64(C.cpu()))
+    # update: every point, through the oracle, on the GPU's assignment
+    C_ref, cnt_ref = oracle_update_chunked(X, ids, C)
     np.testing.assert_array_equal(to_np(counts), cnt_ref)
-    for b in range(2):
-        err = np.linalg.norm(to_np(C_new[b]) - C_ref[b]) / np.linalg.norm(C_ref[b])
-        assert err <= 1e-3
+    assert int(counts.sum()) == B * N
+    Cg = oracle.as_f64(C_new.cpu())
+    for b in range(B):
+        assert np.linalg.norm(Cg[b] - C_ref[b]) <= 1e-3 * np.linalg.norm(C_ref[b])
+    per = np.linalg.norm(Cg - C_ref, axis=-1)
+    scale = np.maximum(np.linalg.norm(C_ref, axis=-1), 1e-3 * np.linalg.norm(C_ref, axis=-1).mean())
+    worst = np.unravel_index(np.argmax(per / scale), per.shape)
+    assert (per <= 1e-3 * scale).all(), f"cluster {worst}: {per[worst] / scale[worst]:.2e}"
+    empty = cnt_ref == 0
+    np.testing.assert_array_equal(Cg[empty], oracle.as_f64(C.cpu())[empty])
+    print(f"workload {idx}: largest cluster {cnt_ref.max()} of {N} points, {int(empty.sum())} empty")
+    # objective: the kernel's full-size inertia against the oracle's distances to the clusters
+    # the kernel chose (this is the inertia of the assignment being checked)
+    ref_in = oracle_inertia_of(X, ids, C, X.dtype)
+    np.testing.assert_allclose(to_np(inertia), ref_in, rtol=1e-4, atol=0)
+    np.testing.assert_allclose(to_np(inertia), to_np(mind.double().sum(1)), rtol=1e-6)
 
 
 def test_rows_workload_full_size(cuda_device):

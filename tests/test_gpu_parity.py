@@ -119,6 +119,38 @@ def test_duplicate_centroids_go_to_lowest_index(dt, d, cuda_device):
     np.testing.assert_array_equal(g[ids_ref == 3], 3)
 
 
+@pytest.mark.parametrize("dt,d,K", [("f16", 128, 300), ("bf16", 128, 300), ("f16", 64, 100),
+                                     ("f16", 256, 60), ("bf16", 8, 300), ("f32", 16, 300)])
+def test_points_on_duplicate_centroids_take_lowest_index(dt, d, K, cuda_device):
+    """Points placed exactly on a centroid that occurs several times: every copy is at distance 0,
+    so the tie rule alone decides, and it must give the lowest index. The copies sit in the same
+    column group of one tile, in other column groups and in other tiles. (The oracle's near-tie
+    exemption covers d2 = 0, so this is asserted directly, not through check_assign.)"""
+    dtype = DT[dt]
+    X, C = mixture(1, 3000, d, K, dtype, cuda_device, seed=17)
+    C = C.to(dtype).float()                  # representable, so a point can equal its centroid
+    groups = {3: [4, 40 % K, 130 % K, (K - 10)], (K // 3): [K // 3 + 1, K // 3 + 20]}
+    for lo, dups in groups.items():
+        for k in dups:
+            if k != lo:
+                C[0, k] = C[0, lo]
+    g = torch.Generator().manual_seed(23)
+    pos = torch.randperm(3000, generator=g)[:600].to(cuda_device)
+    owner = torch.tensor(list(groups), device=cuda_device)[torch.arange(600, device=cuda_device) % 2]
+    X[0, pos] = C[0, owner].to(dtype)
+    Cx, cn = km.km_prep(C, dtype)
+    ids, mind, _ = km.km_assign(X, Cx, cn, want_mind=True)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(to_np(ids[0, pos]), to_np(owner))
+    # the same bound as every other distance check: 1e-5 (||x||^2 + ||c||^2), here 2e-5 ||x||^2
+    xn = (X[0, pos].float() ** 2).sum(-1)
+    assert bool((mind[0, pos] <= 2e-5 * xn + 1e-30).all())
+    # the labels-only form takes the same decisions
+    ids2, _, _ = km.km_assign(X, Cx, cn)
+    torch.cuda.synchronize()
+    assert torch.equal(ids2, ids)
+
+
 def test_all_points_identical(cuda_device):
     X = torch.full((1, 700, 128), 0.5, dtype=torch.float16, device=cuda_device)
     C = torch.randn((1, 300, 128), device=cuda_device)

@@ -20,41 +20,39 @@ pytestmark = pytest.mark.gpu
 KM_ERR_WORKSPACE = 3
 
 
-def _call_noalloc(X, ids, C_prev, w, K):
+def _call_noalloc(X, ids, C_prev, w, C_new, counts, wsum):
     B, N, d = X.shape
-    C_new = torch.empty_like(C_prev)
-    counts = torch.empty((B, K), dtype=torch.int32, device=X.device)
-    wsum = torch.empty((B, K), dtype=torch.float32, device=X.device)
+    K = C_prev.shape[1]
     P = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
-    st = km._load().km_update_noalloc(
+    return km._load().km_update_noalloc(
         P(X), km._dt(X.dtype), P(ids), P(w), B, N, K, d, P(C_prev), P(C_new), P(counts), P(wsum),
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
-    return st, C_new, counts, wsum
 
 
 def test_noalloc_update_matches_workspace_update_twice(cuda_device):
     torch.cuda.set_device(cuda_device)
     cases = [(torch.float16, 2, 3000, 300, 128, True), (torch.float32, 3, 1000, 50, 12, False)]
-    free_after_first = None
     for i, (dtype, B, N, K, d, weighted) in enumerate(cases):
         X, C = mixture(B, N, d, K, dtype, cuda_device, seed=100 + i)
         w = (torch.rand((B, N), device=cuda_device) + 0.05) if weighted else None
         Cx, cn = km.km_prep(C, dtype)
         ids, _, _ = km.km_assign(X, Cx, cn)
         C_ref, counts_ref, wsum_ref = km.km_update(X, ids, C, w=w, want_wsum=True)
+        # outputs are the caller's; they exist before the call is measured
+        C_new = torch.empty_like(C)
+        counts = torch.empty((B, K), dtype=torch.int32, device=cuda_device)
+        wsum = torch.empty((B, K), dtype=torch.float32, device=cuda_device)
         torch.cuda.synchronize()
-        st, C_new, counts, wsum = _call_noalloc(X, ids, C, w, K)
+        free_before = torch.cuda.mem_get_info(cuda_device)[0]
+        st = _call_noalloc(X, ids, C, w, C_new, counts, wsum)
+        torch.cuda.synchronize()
+        free_after = torch.cuda.mem_get_info(cuda_device)[0]
         assert st == 0, km.km_status_string(st)
-        torch.cuda.synchronize()
+        # the call itself took no device memory
+        assert free_after == free_before
         assert torch.equal(counts, counts_ref)
         torch.testing.assert_close(C_new, C_ref, rtol=1e-5, atol=1e-6)
         torch.testing.assert_close(wsum, wsum_ref, rtol=1e-5, atol=1e-6)
-        free = torch.cuda.mem_get_info(cuda_device)[0]
-        if free_after_first is None:
-            free_after_first = free
-        else:
-            # the second call took no device memory beyond what the first one left
-            assert free >= free_after_first
     assert km.km_device_error() == 0
 
 
