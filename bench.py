@@ -10,11 +10,11 @@ larger than the 126 MB L2, so no flush is needed between steps.
   python bench.py --workload {tiny_exact,rows_weighted_1d,large_k_assign,contention_update,
                               contention_update_zipf,emeans,codebook1d} [--gpus N]
 
-A step on the GPU = km_assign (tensor-core FlashAssign; the labels, which is all a Lloyd
-iteration needs: the per-point distance and the inertia are optional outputs) +
-km_update_partial (histogram, scan, scatter, segmented reduce) + km_finalize (the division, with
-the rounded centroids and their norms for the next assignment written by the same kernel):
-exactly one iteration of km_fit's loop without the objective. The assignment with the inertia
+A step on the GPU = km_assign (tensor-core FlashAssign; the labels and the per-cluster counts,
+which is all a Lloyd iteration needs: the per-point distance and the inertia are optional
+outputs) + km_update_next (scan, scatter, then the segmented reduce with the division fused in,
+writing the new centroids, their rounding and norms for the next assignment): exactly one
+iteration of km_fit's loop without the objective. The assignment with the inertia
 requested is timed separately and reported as "assign_with_inertia_ms".
 
 Timing: W untimed warm-up steps, then blocks of exactly K steps, each bracketed by a barrier and
@@ -64,7 +64,7 @@ def update_bytes(Bw, Nw, Dw, esize):
 
 
 UPDATE_BYTES = update_bytes(B, N, D, 2)
-LAUNCHES_PER_STEP = 7   # caug, assign_tc, hist, scan, scatter, segreduce, finalize
+LAUNCHES_PER_STEP = 5   # caug, assign_tc (+ counts), scan_final, scatter, segreduce_final
 MIN_TIMED_S = 0.5
 
 
@@ -341,17 +341,16 @@ def run_gpu(args):
     ws_u = km.workspace(km.KM_OP_UPDATE, B, N, K, D, X.dtype, dev)
     ids = torch.empty((B, N), dtype=torch.int32, device=dev)
     counts = torch.empty((B, K), dtype=torch.int32, device=dev)
-    sums = torch.empty((B, K, D), dtype=torch.float32, device=dev)
     inertia = torch.empty((B,), dtype=torch.float64, device=dev)
     Cx, cn = km.km_prep(C, X.dtype)
     stream = torch.cuda.current_stream()
 
     def assign():
-        km.km_assign(X, Cx, cn, ids=ids, ws=ws_a, stream=stream)
+        km.km_assign(X, Cx, cn, ids=ids, counts=counts, ws=ws_a, stream=stream)
 
     def update():
-        km.km_update_partial(X, ids, K, sums=sums, counts=counts, ws=ws_u, stream=stream)
-        km.km_finalize(sums, counts, C, C_new=C, Cx=Cx, cn=cn, stream=stream)
+        km.km_update_next(X, ids, C, Cx, cn, C_new=C, counts=counts, counts_ready=True, ws=ws_u,
+                          stream=stream)
 
     for _ in range(args.warmup):
         assign()
@@ -615,13 +614,11 @@ def run_workload(args):
         Kw = C.shape[1]
         ws_u = km.workspace(km.KM_OP_UPDATE, Bw, Nw, Kw, Dw, X.dtype, dev)
         counts = torch.empty((Bw, Kw), dtype=torch.int32, device=dev)
-        sums = torch.empty((Bw, Kw, Dw), dtype=torch.float32, device=dev)
         C_new = torch.empty_like(C)
         Cx, cn = km.km_prep(C, X.dtype)
 
-        def update():
-            km.km_update_partial(X, ids, Kw, sums=sums, counts=counts, ws=ws_u, stream=stream)
-            km.km_finalize(sums, counts, C, C_new=C_new, Cx=Cx, cn=cn, stream=stream)
+        def update():   # the histogram of the labels is part of this update
+            km.km_update_next(X, ids, C, Cx, cn, C_new=C_new, counts=counts, ws=ws_u, stream=stream)
 
         for _ in range(args.warmup):
             update()
@@ -637,11 +634,11 @@ def run_workload(args):
                                               "mixture's Zipf(1.1) component labels",
                                   "B": Bw, "N": Nw, "K": Kw, "d": Dw, "largest_segment_frac": largest,
                                   "l2": "inputs larger than L2"},
-                          roofline={"bound": "hbm", "kernel": "hist+scan+scatter+segreduce+finalize",
+                          roofline={"bound": "hbm", "kernel": "hist+scan_final+scatter+segreduce_final",
                                     "achieved": ubytes / (u_ms * 1e-3) / 1e9, "peak": peak_bw, "unit": "GB/s",
                                     "frac": ubytes / (u_ms * 1e-3) / 1e9 / peak_bw,
                                     "algorithmic_bytes": ubytes, "peak_source": peak_kind},
-                          gpu_launches=5 * args.steps * blocks,
+                          gpu_launches=4 * args.steps * blocks,
                           cpu_baseline=dict(cpu_desc, value=ubytes / cpu_s / 1e9, unit="GB/s"),
                           clocks=clk.summary(), device_error=km.km_device_error()))
     else:
@@ -653,15 +650,14 @@ def run_workload(args):
         ws_u = km.workspace(km.KM_OP_UPDATE, Bw, Nw, Kw, Dw, X.dtype, dev)
         ids = torch.empty((Bw, Nw), dtype=torch.int32, device=dev)
         counts = torch.empty((Bw, Kw), dtype=torch.int32, device=dev)
-        sums = torch.empty((Bw, Kw, Dw), dtype=torch.float32, device=dev)
         Cx, cn = km.km_prep(C, X.dtype)
 
         def assign():
-            km.km_assign(X, Cx, cn, ids=ids, ws=ws_a, stream=stream)
+            km.km_assign(X, Cx, cn, ids=ids, counts=counts, ws=ws_a, stream=stream)
 
         def update():
-            km.km_update_partial(X, ids, Kw, sums=sums, counts=counts, ws=ws_u, stream=stream)
-            km.km_finalize(sums, counts, C, C_new=C, Cx=Cx, cn=cn, stream=stream)
+            km.km_update_next(X, ids, C, Cx, cn, C_new=C, counts=counts, counts_ready=True, ws=ws_u,
+                              stream=stream)
 
         for _ in range(args.warmup):
             assign()

@@ -16,7 +16,8 @@ import torch
 __all__ = [
     "KMError", "KM_OP_ASSIGN", "KM_OP_UPDATE", "KM_OP_FIT", "KM_OP_FIT_HOST", "lib_path",
     "km_abi_version", "km_status_string", "km_workspace_size", "km_prep", "km_assign",
-    "km_update", "km_update_partial", "km_finalize", "km_init_grid1d", "km_fit", "km_fit_host",
+    "km_update", "km_update_next", "km_update_partial", "km_finalize", "km_init_grid1d", "km_fit",
+    "km_fit_host",
     "km_device_error", "km_assign_uses_tensor_cores", "workspace",
 ]
 
@@ -52,8 +53,9 @@ def _load():
         "km_abi_version": ([], I),
         "km_workspace_size": ([I, I64, I64, I64, I64, I, I, I], SZ),
         "km_prep": ([P, I, I64, I64, I64, P, P, P], I),
-        "km_assign": ([P, I, P, P, P, I64, I64, I64, I64, P, P, P, P, SZ, P], I),
+        "km_assign": ([P, I, P, P, P, I64, I64, I64, I64, P, P, P, P, P, SZ, P], I),
         "km_update": ([P, I, P, P, I64, I64, I64, I64, P, P, P, P, P, SZ, P], I),
+        "km_update_next": ([P, I, P, P, I64, I64, I64, I64, P, P, P, P, P, I, P, P, SZ, P], I),
         "km_update_partial": ([P, I, P, P, I64, I64, I64, I64, P, P, P, P, SZ, P], I),
         "km_finalize": ([P, P, P, P, I64, I64, I64, P, I, P, P, P], I),
         "km_init_grid1d": ([P, I, I64, I64, I64, P, P], I),
@@ -144,8 +146,9 @@ def km_prep(C, dtype, Cx=None, cn=None, stream=None):
 
 
 def km_assign(X, Cx, cn=None, w=None, ids=None, mind=None, inertia=None, want_mind=False,
-              want_inertia=False, ws=None, stream=None):
-    """Assignment stage. X: [B,N,d], Cx: [B,K,d] same dtype. Returns (ids, mind, inertia)."""
+              want_inertia=False, counts=None, ws=None, stream=None):
+    """Assignment stage. X: [B,N,d], Cx: [B,K,d] same dtype. Returns (ids, mind, inertia).
+    `counts` ([B,K] int32, optional) receives the number of points assigned to each cluster."""
     B, N, d = X.shape
     K = Cx.shape[1]
     dev = X.device
@@ -159,11 +162,12 @@ def km_assign(X, Cx, cn=None, w=None, ids=None, mind=None, inertia=None, want_mi
     if want_inertia and inertia is None:
         inertia = torch.empty((B,), dtype=torch.float64, device=dev)
     _need(ids, "ids", torch.int32, (B, N), dev)
+    _need(counts, "counts", torch.int32, (B, K), dev)
     if ws is None:
         ws = workspace(KM_OP_ASSIGN, B, N, K, d, X.dtype, dev)
     _check("km_assign", _load().km_assign(
         _p(X), _dt(X.dtype), _p(Cx), _p(cn), _p(w), B, N, K, d, _p(ids), _p(mind), _p(inertia),
-        _p(ws), ws.numel(), _s(stream)))
+        _p(counts), _p(ws), ws.numel(), _s(stream)))
     return ids, mind, inertia
 
 
@@ -186,6 +190,34 @@ def km_update(X, ids, C_prev, w=None, C_new=None, counts=None, wsum=None, want_w
     _check("km_update", _load().km_update(
         _p(X), _dt(X.dtype), _p(ids), _p(w), B, N, K, d, _p(C_prev), _p(C_new), _p(counts),
         _p(wsum), _p(ws), ws.numel(), _s(stream)))
+    return C_new, counts, wsum
+
+
+def km_update_next(X, ids, C_prev, Cx, cn, w=None, C_new=None, counts=None, wsum=None,
+                   want_wsum=False, counts_ready=False, ws=None, stream=None):
+    """Update stage that also writes the next assignment's inputs: Cx (C_new rounded to X's
+    dtype) and cn = ||Cx||^2, both given by the caller. With counts_ready the given `counts`
+    already hold the histogram of ids (km_assign(counts=...)). Returns (C_new, counts, wsum)."""
+    B, N, d = X.shape
+    K = C_prev.shape[1]
+    dev = X.device
+    _need(X, "X")
+    _need(ids, "ids", torch.int32, (B, N), dev)
+    _need(C_prev, "C_prev", torch.float32, (B, K, d), dev)
+    _need(Cx, "Cx", X.dtype, (B, K, d), dev)
+    _need(cn, "cn", torch.float32, (B, K), dev)
+    _need(w, "w", torch.float32, (B, N), dev)
+    C_new = torch.empty_like(C_prev) if C_new is None else C_new
+    if counts_ready and counts is None:
+        raise ValueError("counts_ready needs the counts")
+    counts = torch.empty((B, K), dtype=torch.int32, device=dev) if counts is None else counts
+    if want_wsum and wsum is None:
+        wsum = torch.empty((B, K), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(KM_OP_UPDATE, B, N, K, d, X.dtype, dev)
+    _check("km_update_next", _load().km_update_next(
+        _p(X), _dt(X.dtype), _p(ids), _p(w), B, N, K, d, _p(C_prev), _p(C_new), _p(Cx), _p(cn),
+        _p(counts), int(bool(counts_ready)), _p(wsum), _p(ws), ws.numel(), _s(stream)))
     return C_new, counts, wsum
 
 

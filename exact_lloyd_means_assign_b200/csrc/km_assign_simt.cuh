@@ -21,7 +21,8 @@ template <typename T>
 __global__ void __launch_bounds__(kSimtPts)
     assign_simt_kernel(const T *__restrict__ X, const T *__restrict__ Cx,
                        const float *__restrict__ w, int N, int K, int d, int32_t *__restrict__ ids,
-                       float *__restrict__ mind, double *__restrict__ inertia) {
+                       float *__restrict__ mind, double *__restrict__ inertia,
+                       int32_t *__restrict__ counts) {
     __shared__ float xs[kSimtDC][kSimtPts + 1];
     __shared__ float cs[kSimtKT][kSimtDC];
     __shared__ double red[kSimtPts / 32];
@@ -80,6 +81,12 @@ __global__ void __launch_bounds__(kSimtPts)
         ids[gi] = bi;
         if (mind) mind[gi] = best;
         contrib = static_cast<double>(w ? w[gi] : 1.f) * static_cast<double>(best);
+    }
+    if (counts) {   // per-cluster point counts, one atomic per distinct cluster in the warp
+        const int key = valid ? bi : -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, key);
+        if (key >= 0 && (tid & 31) == __ffs(peers) - 1)
+            atomicAdd(counts + static_cast<int64_t>(b) * K + key, __popc(peers));
     }
     if (inertia) {
         contrib = warp_sum(contrib);

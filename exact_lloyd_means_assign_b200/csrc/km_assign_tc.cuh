@@ -133,6 +133,7 @@ struct Params {
     int32_t *ids;
     float *mind;
     double *inertia;
+    int32_t *counts;   // per-cluster point counts (added to; zeroed by the host), or null
 };
 
 // Upper 32 bits of a K-major shared-memory matrix descriptor (stride byte offset, version 1,
@@ -641,6 +642,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 if (p.inertia) {
                     contrib = warp_sum(contrib);
                     if (lane == 0) atomicAdd(p.inertia + b, contrib);
+                }
+                if (p.counts) {
+                    // the histogram the update's sort starts from: one atomic per distinct
+                    // cluster among the warp's 32 points
+                    const int key = i < p.N ? best_i : -1;
+                    const unsigned peers = __match_any_sync(0xffffffffu, key);
+                    if (key >= 0 && lane == __ffs(peers) - 1)
+                        atomicAdd(p.counts + static_cast<size_t>(b) * p.K + key, __popc(peers));
                 }
             }
         }

@@ -90,6 +90,33 @@ inline UpdateWs carve_update(Carver &c, int64_t B, int64_t N, int64_t K, int64_t
     return u;
 }
 
+// The fused reduce-and-divide form: the sort scratch, arrival counters and the per-range partial
+// slots of split segments (ranges per batch element are at most kFinalWarpsMax / B + 1).
+constexpr int64_t kFinalWarpsMax = 2048;
+struct FinalWs {
+    int32_t *offsets, *cursor, *perm, *arrive;
+    float *slots, *wslots;
+};
+inline int64_t final_rpb_max(int64_t B) { return std::max<int64_t>(1, kFinalWarpsMax / B) + 1; }
+inline FinalWs carve_final(Carver &c, int64_t B, int64_t N, int64_t K, int64_t d) {
+    FinalWs f;
+    f.offsets = c.take<int32_t>(static_cast<size_t>(B * (K + 1)) * 4);
+    f.cursor = c.take<int32_t>(static_cast<size_t>(B * K) * 4);
+    f.perm = c.take<int32_t>(static_cast<size_t>(B * N) * 4);
+    f.arrive = c.take<int32_t>(static_cast<size_t>(B * K) * 4);
+    const int64_t nslots = B * final_rpb_max(B) * 2;
+    f.slots = c.take<float>(static_cast<size_t>(nslots * d) * 4);
+    f.wslots = c.take<float>(static_cast<size_t>(nslots) * 4);
+    return f;
+}
+// bytes that cover both update forms (the caller's workspace serves whichever runs)
+inline size_t ws_update(int64_t B, int64_t N, int64_t K, int64_t d) {
+    Carver a(nullptr), f(nullptr);
+    carve_update(a, B, N, K, d);
+    carve_final(f, B, N, K, d);
+    return std::max(a.off, f.off);
+}
+
 inline bool fit1d_ok(int64_t N, int64_t K, int64_t d) {
     return d == 1 && K <= km::fit1d::KMAX && N <= km::fit1d::NMAX;
 }
@@ -129,11 +156,9 @@ inline FitWs carve_fit(Carver &c, int64_t B, int64_t N, int64_t K, int64_t d, km
     f.counts = c.take<int32_t>(static_cast<size_t>(B * K) * 4);
     f.inertia = c.take<double>(static_cast<size_t>(B) * 8);
     f.rest = c.base ? c.base + c.off : nullptr;
-    Carver u(nullptr);
-    carve_update(u, B, N, K, d);
     Carver g(nullptr);
     if (fit1d_rows_ok(N, K, d)) carve_fit1d(g, B, N);
-    c.off += std::max({u.off, ws_assign(B, K, d, dt), g.off});
+    c.off += std::max({ws_update(B, N, K, d), ws_assign(B, K, d, dt), g.off});
     return f;
 }
 
@@ -264,7 +289,7 @@ km_status finalize_dispatch(const float *sums, const float *wsum, const int32_t 
 template <typename T>
 km_status run_assign_simt(const void *X, const void *Cx, const float *w, int64_t B, int64_t N,
                           int64_t K, int64_t d, int32_t *ids, float *mind, double *inertia,
-                          cudaStream_t st) {
+                          int32_t *counts, cudaStream_t st) {
     const T *Xt = static_cast<const T *>(X);
     const T *Ct = static_cast<const T *>(Cx);
     for (int64_t b0 = 0; b0 < B; b0 += kMaxGridY) {
@@ -273,7 +298,7 @@ km_status run_assign_simt(const void *X, const void *Cx, const float *w, int64_t
         km::assign_simt_kernel<T><<<grid, km::kSimtPts, 0, st>>>(
             Xt + b0 * N * d, Ct + b0 * K * d, w ? w + b0 * N : nullptr, static_cast<int>(N),
             static_cast<int>(K), static_cast<int>(d), ids + b0 * N, mind ? mind + b0 * N : nullptr,
-            inertia ? inertia + b0 : nullptr);
+            inertia ? inertia + b0 : nullptr, counts ? counts + b0 * K : nullptr);
         if (launch_status() != KM_OK) return KM_ERR_CUDA;
     }
     return KM_OK;
@@ -339,7 +364,7 @@ km_status launch_assign_tc(const CUtensorMap &tmX, const CUtensorMap &tmC, const
 template <typename T>
 km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float *cn,
                         const float *w, int64_t B, int64_t N, int64_t K, int64_t d, int32_t *ids,
-                        float *mind, double *inertia, void *caug, cudaStream_t st) {
+                        float *mind, double *inertia, int32_t *counts, void *caug, cudaStream_t st) {
     using namespace km::tc;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return KM_ERR_CUDA;
@@ -405,6 +430,7 @@ km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float 
     p.ids = ids;
     p.mind = mind;
     p.inertia = inertia;
+    p.counts = counts;
     const int64_t items = B * p.mtiles;
     if (items > kMaxIndex) return KM_ERR_UNSUPPORTED;
     // (bn, chunks of 64 along d); bn = 256 with d > 192 never fits (tc_bn narrows it)
@@ -421,23 +447,29 @@ km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float 
 // path can run.
 // With accumulate_inertia the objective is added to `inertia` instead of overwriting it (the
 // streamed fit sums it over chunks of points).
+// counts (optional) receive the per-cluster point counts of the assignment (overwritten).
 km_status do_assign(const void *X, km_dtype dt, const void *Cx, const float *cn, const float *w,
                     int64_t B, int64_t N, int64_t K, int64_t d, int32_t *ids, float *mind,
-                    double *inertia, void *caug, cudaStream_t st, bool accumulate_inertia = false) {
+                    double *inertia, void *caug, cudaStream_t st, bool accumulate_inertia = false,
+                    int32_t *counts = nullptr) {
     if (inertia && !accumulate_inertia &&
         cudaMemsetAsync(inertia, 0, static_cast<size_t>(B) * 8, st) != cudaSuccess)
+        return KM_ERR_CUDA;
+    if (counts && cudaMemsetAsync(counts, 0, static_cast<size_t>(B * K) * 4, st) != cudaSuccess)
         return KM_ERR_CUDA;
     const bool tc = tc_shape_ok(dt, d) && aligned(X, 16) && aligned(Cx, 16) && caug != nullptr &&
                     B * ceil_div(N, 128) <= kMaxIndex;
     if (tc) {
         if (dt == KM_F16)
-            return run_assign_tc<__half>(X, dt, Cx, cn, w, B, N, K, d, ids, mind, inertia, caug, st);
-        return run_assign_tc<__nv_bfloat16>(X, dt, Cx, cn, w, B, N, K, d, ids, mind, inertia, caug, st);
+            return run_assign_tc<__half>(X, dt, Cx, cn, w, B, N, K, d, ids, mind, inertia, counts, caug, st);
+        return run_assign_tc<__nv_bfloat16>(X, dt, Cx, cn, w, B, N, K, d, ids, mind, inertia, counts,
+                                            caug, st);
     }
     switch (dt) {
-        case KM_F32: return run_assign_simt<float>(X, Cx, w, B, N, K, d, ids, mind, inertia, st);
-        case KM_F16: return run_assign_simt<__half>(X, Cx, w, B, N, K, d, ids, mind, inertia, st);
-        default: return run_assign_simt<__nv_bfloat16>(X, Cx, w, B, N, K, d, ids, mind, inertia, st);
+        case KM_F32: return run_assign_simt<float>(X, Cx, w, B, N, K, d, ids, mind, inertia, counts, st);
+        case KM_F16: return run_assign_simt<__half>(X, Cx, w, B, N, K, d, ids, mind, inertia, counts, st);
+        default:
+            return run_assign_simt<__nv_bfloat16>(X, Cx, w, B, N, K, d, ids, mind, inertia, counts, st);
     }
 }
 
@@ -610,6 +642,162 @@ km_status do_update_partial(const void *X, km_dtype dt, const int32_t *ids, cons
     return launch_status();
 }
 
+// ---------------------------------------------------------------- fused update (reduce + divide)
+
+// Rows of d = 32 * V elements of 128, 256 or 512 bytes, 16-byte aligned X, and B * N rows that
+// fit the tensor map's 32-bit row coordinate.
+inline bool final_ok(km_dtype dt, const void *X, int64_t B, int64_t N, int64_t d) {
+    if (d % 32 != 0 || !aligned(X, 16) || B * N >= (int64_t{1} << 31)) return false;
+    const int64_t rb = d * static_cast<int64_t>(dtype_size(dt));
+    return rb == 128 || rb == 256 || rb == 512;
+}
+
+template <typename T, int V, bool WEIGHTED>
+km_status launch_final(const CUtensorMap &tm, km::upd::FinalParams &p, int64_t B, int64_t N,
+                       cudaStream_t st) {
+    using namespace km::upd;
+    constexpr int RB = 32 * V * static_cast<int>(sizeof(T));
+    constexpr int NW = fz_warps(RB);
+    if (cudaFuncSetAttribute(segreduce_final_kernel<T, V, WEIGHTED>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, fz_smem(RB)) != cudaSuccess)
+        return KM_ERR_CUDA;
+    // one CTA per SM; every warp walks one range of sorted positions of one batch element
+    const int64_t total = static_cast<int64_t>(std::min(num_sms(), static_cast<int>(kFinalWarpsMax / NW))) * NW;
+    const int64_t rpb0 = std::max<int64_t>(1, total / B);
+    const int64_t range = std::max<int64_t>(64, ceil_div(ceil_div(N, rpb0), 32) * 32);
+    const int64_t rpb = ceil_div(N, range);
+    if (rpb > final_rpb_max(B)) return KM_ERR_UNSUPPORTED;   // never: rpb <= rpb0
+    p.range = static_cast<int>(range);
+    p.rpb = static_cast<int>(rpb);
+    const int64_t warps = B * rpb;
+    segreduce_final_kernel<T, V, WEIGHTED>
+        <<<static_cast<unsigned>(ceil_div(warps, NW)), NW * 32, fz_smem(RB), st>>>(tm, p);
+    return launch_status();
+}
+
+template <typename T, int V>
+km_status final_weighted(const CUtensorMap &tm, km::upd::FinalParams &p, int64_t B, int64_t N,
+                         cudaStream_t st) {
+    return p.w ? launch_final<T, V, true>(tm, p, B, N, st) : launch_final<T, V, false>(tm, p, B, N, st);
+}
+
+// One sort-inverse update that writes the new centroids directly (no per-cluster sums array):
+// counts (overwritten), then C_new and, when given, Cx (X's dtype), cn and wsum. Requires
+// final_ok(); `ws` holds carve_final's layout.
+template <typename T>
+km_status run_update_final(const void *X, km_dtype dt, const int32_t *ids, const float *w,
+                           int64_t B, int64_t N, int64_t K, int64_t d, const float *C_prev,
+                           float *C_new, void *Cx, float *cn, int32_t *counts, bool have_counts,
+                           float *wsum, void *ws, cudaStream_t st) {
+    using namespace km::upd;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return KM_ERR_CUDA;
+    Carver c(ws);
+    const FinalWs f = carve_final(c, B, N, K, d);
+    if (!have_counts && cudaMemsetAsync(counts, 0, static_cast<size_t>(B * K) * 4, st) != cudaSuccess)
+        return KM_ERR_CUDA;
+    const bool smem_bins = K <= SMEM_K_MAX;
+    const int64_t ntiles = ceil_div(N, TILE);
+    if (cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_K_MAX * 4) != cudaSuccess ||
+        cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (SMEM_K_MAX + TILE) * 4) != cudaSuccess)
+        return KM_ERR_CUDA;
+    for (int64_t b0 = 0; b0 < B && !have_counts; b0 += kMaxGridY) {
+        const int64_t nb = std::min<int64_t>(kMaxGridY, B - b0);
+        dim3 grid(static_cast<unsigned>(ntiles), static_cast<unsigned>(nb));
+        hist_kernel<<<grid, TILE_THREADS, smem_bins ? K * 4 : 0, st>>>(
+            ids + b0 * N, static_cast<int>(N), static_cast<int>(K), counts + b0 * K, smem_bins);
+        if (launch_status() != KM_OK) return KM_ERR_CUDA;
+    }
+    scan_final_kernel<T><<<static_cast<unsigned>(B), SCAN_THREADS, 0, st>>>(
+        counts, static_cast<int>(K), static_cast<int>(d), f.offsets, f.cursor, f.arrive, C_prev,
+        C_new, static_cast<T *>(Cx), cn, wsum);
+    if (launch_status() != KM_OK) return KM_ERR_CUDA;
+    const size_t scatter_smem = smem_bins ? static_cast<size_t>(K + TILE) * 4 : 0;
+    for (int64_t b0 = 0; b0 < B; b0 += kMaxGridY) {
+        const int64_t nb = std::min<int64_t>(kMaxGridY, B - b0);
+        dim3 grid(static_cast<unsigned>(ntiles), static_cast<unsigned>(nb));
+        scatter_kernel<<<grid, TILE_THREADS, scatter_smem, st>>>(
+            ids + b0 * N, static_cast<int>(N), static_cast<int>(K), f.cursor + b0 * K,
+            f.perm + b0 * N, smem_bins);
+        if (launch_status() != KM_OK) return KM_ERR_CUDA;
+    }
+    // X as [B*N rows, d] with one-row boxes for the four-row gathers
+    CUtensorMap tm;
+    const CUtensorMapDataType tdt = dt == KM_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                    : dt == KM_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                   : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(B * N)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * dtype_size(dt)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(d), 1};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&tm, tdt, 2, const_cast<void *>(X), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return KM_ERR_CUDA;
+    FinalParams p;
+    p.B = static_cast<int>(B);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.range = 0;
+    p.rpb = 0;
+    p.perm = f.perm;
+    p.offsets = f.offsets;
+    p.w = w;
+    p.C_prev = C_prev;
+    p.C_new = C_new;
+    p.Cx = Cx;
+    p.cn = cn;
+    p.wsum = wsum;
+    p.slots = f.slots;
+    p.wslots = f.wslots;
+    p.arrive = f.arrive;
+    constexpr int VV = static_cast<int>(16 / sizeof(T));   // 16-byte rows per lane at most
+    const int64_t V = d / 32;
+    if (V == VV) return final_weighted<T, VV>(tm, p, B, N, st);
+    if (V == VV / 2) return final_weighted<T, VV / 2>(tm, p, B, N, st);
+    if (V == VV / 4) return final_weighted<T, VV / 4>(tm, p, B, N, st);
+    return KM_ERR_UNSUPPORTED;
+}
+
+km_status update_final_dispatch(const void *X, km_dtype dt, const int32_t *ids, const float *w,
+                                int64_t B, int64_t N, int64_t K, int64_t d, const float *C_prev,
+                                float *C_new, void *Cx, float *cn, int32_t *counts, bool have_counts,
+                                float *wsum, void *ws, cudaStream_t st) {
+    switch (dt) {
+        case KM_F32:
+            return run_update_final<float>(X, dt, ids, w, B, N, K, d, C_prev, C_new, Cx, cn, counts,
+                                           have_counts, wsum, ws, st);
+        case KM_F16:
+            return run_update_final<__half>(X, dt, ids, w, B, N, K, d, C_prev, C_new, Cx, cn, counts,
+                                            have_counts, wsum, ws, st);
+        default:
+            return run_update_final<__nv_bfloat16>(X, dt, ids, w, B, N, K, d, C_prev, C_new, Cx, cn,
+                                                   counts, have_counts, wsum, ws, st);
+    }
+}
+
+// The whole update: the fused form where it applies, else the sums array and finalize_kernel.
+// `ws` holds ws_update() bytes. wsum (optional) receives the per-cluster weight sums. With
+// have_counts the counts already hold the histogram of ids (the assignment wrote it) and the
+// fused form skips its own histogram pass.
+km_status do_update(const void *X, km_dtype dt, const int32_t *ids, const float *w, int64_t B,
+                    int64_t N, int64_t K, int64_t d, const float *C_prev, float *C_new,
+                    km_dtype cx_dt, void *Cx, float *cn, int32_t *counts, float *wsum, void *ws,
+                    cudaStream_t st, bool have_counts = false) {
+    if (final_ok(dt, X, B, N, d) && (!Cx || cx_dt == dt))
+        return update_final_dispatch(X, dt, ids, w, B, N, K, d, C_prev, C_new, Cx, cn, counts,
+                                     have_counts, wsum, ws, st);
+    Carver r(ws);
+    UpdateWs u = carve_update(r, B, N, K, d);
+    float *ws_w = wsum ? wsum : (w ? u.wsum : nullptr);
+    km_status s = do_update_partial(X, dt, ids, w, B, N, K, d, u.sums, ws_w, counts, u, st);
+    if (s != KM_OK) return s;
+    return finalize_dispatch(u.sums, w ? ws_w : nullptr, counts, C_prev, B * K, d, C_new,
+                             Cx ? cx_dt : KM_F32, Cx, cn, st);
+}
+
 template <typename T>
 km_status run_fit1d(const void *X, const float *w, int64_t B, int64_t N, int64_t K, float *C,
                     int iters, int32_t *ids, double *inertia_hist, float *C_hist, void *ws,
@@ -658,8 +846,6 @@ km_status do_fit(const void *X, km_dtype dt, const float *w, int64_t B, int64_t 
                 return run_fit1d<__nv_bfloat16>(X, w, B, N, K, C, iters, ids, inertia_hist, C_hist, f.rest, st);
         }
     }
-    Carver r(f.rest);
-    UpdateWs u = carve_update(r, B, N, K, d);
     void *caug = f.rest;  // assignment scratch shares the update region (used one after the other)
     const size_t cbytes = static_cast<size_t>(B * K * d) * 4;
     km_status s = prep_dispatch(C, dt, B * K, d, f.Cx, f.cn, st);
@@ -669,11 +855,10 @@ km_status do_fit(const void *X, km_dtype dt, const float *w, int64_t B, int64_t 
                                       cudaMemcpyDeviceToDevice, st) != cudaSuccess)
             return KM_ERR_CUDA;
         double *in = inertia_hist ? inertia_hist + static_cast<int64_t>(t) * B : nullptr;
-        s = do_assign(X, dt, f.Cx, f.cn, w, B, N, K, d, f.ids, nullptr, in, caug, st);
+        s = do_assign(X, dt, f.Cx, f.cn, w, B, N, K, d, f.ids, nullptr, in, caug, st, false, f.counts);
         if (s != KM_OK) return s;
-        s = do_update_partial(X, dt, f.ids, w, B, N, K, d, u.sums, w ? u.wsum : nullptr, f.counts, u, st);
-        if (s != KM_OK) return s;
-        s = finalize_dispatch(u.sums, w ? u.wsum : nullptr, f.counts, C, B * K, d, C, dt, f.Cx, f.cn, st);
+        s = do_update(X, dt, f.ids, w, B, N, K, d, C, C, dt, f.Cx, f.cn, f.counts, nullptr, f.rest, st,
+                      true);
         if (s != KM_OK) return s;
     }
     if (C_hist && cudaMemcpyAsync(C_hist + static_cast<int64_t>(iters) * B * K * d, C, cbytes,
@@ -915,7 +1100,7 @@ const char *km_status_string(km_status s) {
     return "KM_ERR_UNKNOWN";
 }
 
-int km_abi_version(void) { return 1; }
+int km_abi_version(void) { return 2; }
 
 int km_assign_uses_tensor_cores(km_dtype dtype, int64_t d, const void *X, const void *Cx) {
     return valid_dtype(dtype) && tc_shape_ok(dtype, d) && aligned(X, 16) && aligned(Cx, 16) ? 1 : 0;
@@ -927,7 +1112,7 @@ size_t km_workspace_size(km_op op, int64_t B, int64_t N, int64_t K, int64_t d, k
     Carver c(nullptr);
     switch (op) {
         case KM_OP_ASSIGN: return ws_assign(B, K, d, dtype);
-        case KM_OP_UPDATE: carve_update(c, B, N, K, d); return c.off;
+        case KM_OP_UPDATE: return ws_update(B, N, K, d);
         case KM_OP_FIT: carve_fit(c, B, N, K, d, dtype); return c.off;
         case KM_OP_FIT_HOST: carve_host(c, B, N, K, d, dtype, weighted != 0, iters); return c.off;
     }
@@ -944,16 +1129,16 @@ km_status km_prep(const float *C, km_dtype dtype, int64_t B, int64_t K, int64_t 
 
 km_status km_assign(const void *X, km_dtype dtype, const void *Cx, const float *cn, const float *w,
                     int64_t B, int64_t N, int64_t K, int64_t d, int32_t *ids, float *mind,
-                    double *inertia, void *ws, size_t ws_bytes, void *stream) {
+                    double *inertia, int32_t *counts, void *ws, size_t ws_bytes, void *stream) {
     if (!X || !Cx || !ids || !valid_dtype(dtype) || !sizes_ok(B, N, K, d) ||
         !elem_aligned(X, dtype) || !elem_aligned(Cx, dtype) || !aligned(ids, 4) ||
         (w && !aligned(w, 4)) || (cn && !aligned(cn, 4)) || (mind && !aligned(mind, 4)) ||
-        (inertia && !aligned(inertia, 8)))
+        (inertia && !aligned(inertia, 8)) || (counts && !aligned(counts, 4)))
         return KM_ERR_INVALID_ARG;
     const size_t need = ws_assign(B, K, d, dtype);
     if (need && (!ws || ws_bytes < need || !aligned(ws, kAlign))) return KM_ERR_WORKSPACE;
     return do_assign(X, dtype, Cx, cn, w, B, N, K, d, ids, mind, inertia, need ? ws : nullptr,
-                     S(stream));
+                     S(stream), false, counts);
 }
 
 km_status km_update_partial(const void *X, km_dtype dtype, const int32_t *ids, const float *w,
@@ -988,16 +1173,23 @@ km_status km_update(const void *X, km_dtype dtype, const int32_t *ids, const flo
         !elem_aligned(X, dtype) || !aligned(ids, 4) || !aligned(counts, 4) || !aligned(C_prev, 4) ||
         !aligned(C_new, 4) || (w && !aligned(w, 4)) || (wsum && !aligned(wsum, 4)))
         return KM_ERR_INVALID_ARG;
-    Carver c(nullptr);
-    carve_update(c, B, N, K, d);
-    if (!ws || ws_bytes < c.off || !aligned(ws, kAlign)) return KM_ERR_WORKSPACE;
-    Carver r(ws);
-    UpdateWs u = carve_update(r, B, N, K, d);
-    float *ws_w = wsum ? wsum : (w ? u.wsum : nullptr);
-    km_status s = do_update_partial(X, dtype, ids, w, B, N, K, d, u.sums, ws_w, counts, u, S(stream));
-    if (s != KM_OK) return s;
-    return finalize_dispatch(u.sums, w ? ws_w : nullptr, counts, C_prev, B * K, d, C_new, KM_F32,
-                             nullptr, nullptr, S(stream));
+    if (!ws || ws_bytes < ws_update(B, N, K, d) || !aligned(ws, kAlign)) return KM_ERR_WORKSPACE;
+    return do_update(X, dtype, ids, w, B, N, K, d, C_prev, C_new, KM_F32, nullptr, nullptr, counts,
+                     wsum, ws, S(stream));
+}
+
+km_status km_update_next(const void *X, km_dtype dtype, const int32_t *ids, const float *w,
+                         int64_t B, int64_t N, int64_t K, int64_t d, const float *C_prev,
+                         float *C_new, void *Cx, float *cn, int32_t *counts, int counts_ready,
+                         float *wsum, void *ws, size_t ws_bytes, void *stream) {
+    if (!X || !ids || !C_prev || !C_new || !Cx || !cn || !counts || !valid_dtype(dtype) ||
+        !sizes_ok(B, N, K, d) || !elem_aligned(X, dtype) || !aligned(ids, 4) || !aligned(counts, 4) ||
+        !aligned(C_prev, 4) || !aligned(C_new, 4) || !elem_aligned(Cx, dtype) || !aligned(cn, 4) ||
+        (w && !aligned(w, 4)) || (wsum && !aligned(wsum, 4)))
+        return KM_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < ws_update(B, N, K, d) || !aligned(ws, kAlign)) return KM_ERR_WORKSPACE;
+    return do_update(X, dtype, ids, w, B, N, K, d, C_prev, C_new, dtype, Cx, cn, counts, wsum, ws,
+                     S(stream), counts_ready != 0);
 }
 
 km_status km_init_grid1d(const void *X, km_dtype dtype, int64_t B, int64_t N, int64_t K, float *C,

@@ -439,5 +439,417 @@ __global__ void __launch_bounds__(ROWS_THREADS, ROWS_BLOCKS_PER_SM)
     if (acck >= 0) flush(acck);
 }
 
+// ------------------------------------------------------------------ reduce and divide in one pass
+//
+// segreduce_final_kernel is the segmented reduction above fused with the final divide, for
+// d = 32 * V with rows of 128, 256 or 512 bytes. Two differences from segreduce_rows_kernel:
+//
+// Row gathers go through the tensor-memory-access engine: each warp owns a ring of S stages of
+// 32 rows in shared memory, and for every chunk of 32 sorted positions eight of its lanes issue
+// one four-row gather each (cp.async.bulk.tensor tile::gather4 on a [B*N, d] view of X, box one
+// row high), completing on the stage's mbarrier. S - 1 chunks are in flight while the warp sums
+// the current one out of shared memory, so the bytes in flight are bounded by shared memory,
+// not by registers (the register-staged form is bound by gather latency).
+//
+// No per-cluster sums array: a run that lies entirely inside the warp's range of sorted positions
+// is a whole cluster, so the warp divides it by its count (or weight sum) and writes C_new, and
+// when asked the rounded Cx, ||Cx||^2 and the weight sum. A cluster whose segment crosses range
+// boundaries leaves one partial per range it touches in a per-range slot (side 0: the range's
+// first run, side 1: its last run), then counts itself on the cluster's arrival counter; the
+// warp that arrives last (the count of ranges touching the segment is known from the offsets)
+// adds the partials in range order and finalizes. Nobody waits, so there is no spin. Empty
+// clusters are written by scan_final_kernel.
+constexpr int FZ_CHUNK = 32;
+
+struct FinalParams {
+    int B, N, K, range, rpb;
+    const int32_t *perm, *offsets;
+    const float *w;
+    const float *C_prev;
+    float *C_new;
+    void *Cx;
+    float *cn;
+    float *wsum;        // per-cluster weight sums out (counts when unweighted), or null
+    float *slots;       // [B * rpb * 2, d] partials of split segments
+    float *wslots;      // [B * rpb * 2] their weight sums
+    int32_t *arrive;    // [B, K] arrival counters, zeroed by scan_final_kernel
+};
+
+// warps per CTA and ring depth for a row of RB bytes (one CTA per SM, 192 KB of rings). The
+// summing loop is bound by the latency of its own instruction chains, so the rings favour more
+// warps over deeper rings (measured: 12 warps x 2 stages of 32 rows beat 8 x 3 for 256-byte rows).
+__host__ __device__ constexpr int fz_warps(int RB) { return RB >= 512 ? 6 : (RB >= 256 ? 12 : 16); }
+__host__ __device__ constexpr int fz_stages(int RB) { return RB >= 128 && RB < 256 ? 3 : 2; }
+__host__ __device__ constexpr int fz_smem(int RB) {
+    return fz_warps(RB) * fz_stages(RB) * FZ_CHUNK * RB + 1024;
+}
+
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *tm, uint32_t bar, int col,
+                                            int r0, int r1, int r2, int r3, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(dst),
+        "l"(tm), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+template <typename T, int V> struct RowLd;
+template <typename T> struct RowLd<T, 2> { using U = uint32_t; };     // 16-bit V=2: 4 B
+template <> struct RowLd<float, 1> { using U = float; };
+template <typename T> struct RowLd<T, 4> { using U = uint2; };
+template <> struct RowLd<float, 2> { using U = float2; };
+template <typename T> struct RowLd<T, 8> { using U = uint4; };
+template <> struct RowLd<float, 4> { using U = float4; };
+
+// The V elements lane `lane` owns of one row in shared memory, as fp32.
+template <typename T, int V>
+__device__ __forceinline__ void row_vals(const uint8_t *row, int lane, float (&x)[V]) {
+    using U = typename RowLd<T, V>::U;
+    const U u = reinterpret_cast<const U *>(row)[lane];
+    const T *t = reinterpret_cast<const T *>(&u);
+#pragma unroll
+    for (int e = 0; e < V; ++e) x[e] = Cvt<T>::to_f(t[e]);
+}
+
+// acc += the V elements lane `lane` owns of one row. For 16-bit rows a mixed-precision FMA
+// (x * 1 + acc in fp32, the product exact) adds each element without a separate conversion.
+template <typename T> __device__ __forceinline__ float add_lo_hi(uint32_t w, float &hi_acc, float lo_acc);
+template <> __device__ __forceinline__ float add_lo_hi<__half>(uint32_t w, float &hi_acc, float lo_acc) {
+    asm("{\n\t.reg .b16 l, h, one;\n\tmov.b32 {l, h}, %2;\n\tmov.b16 one, 0x3C00;\n\t"
+        "fma.rn.f32.f16 %0, l, one, %0;\n\tfma.rn.f32.f16 %1, h, one, %1;\n\t}"
+        : "+f"(lo_acc), "+f"(hi_acc) : "r"(w));
+    return lo_acc;
+}
+template <> __device__ __forceinline__ float add_lo_hi<__nv_bfloat16>(uint32_t w, float &hi_acc, float lo_acc) {
+    asm("{\n\t.reg .b16 l, h, one;\n\tmov.b32 {l, h}, %2;\n\tmov.b16 one, 0x3F80;\n\t"
+        "fma.rn.f32.bf16 %0, l, one, %0;\n\tfma.rn.f32.bf16 %1, h, one, %1;\n\t}"
+        : "+f"(lo_acc), "+f"(hi_acc) : "r"(w));
+    return lo_acc;
+}
+template <typename T, int V>
+__device__ __forceinline__ void row_add(const uint8_t *row, int lane, float (&acc)[V]) {
+    if constexpr (sizeof(T) == 2) {
+        using U = typename RowLd<T, V>::U;
+        const U u = reinterpret_cast<const U *>(row)[lane];
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(&u);
+#pragma unroll
+        for (int e = 0; e < V / 2; ++e) acc[2 * e] = add_lo_hi<T>(w[e], acc[2 * e + 1], acc[2 * e]);
+    } else {
+        float x[V];
+        row_vals<T, V>(row, lane, x);
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[e] += x[e];
+    }
+}
+
+// C_new (and optionally Cx, ||Cx||^2, the weight sum) of cluster row `row` from its sums.
+template <typename T, int V>
+__device__ __forceinline__ void finalize_one(const FinalParams &p, int64_t row, int lane,
+                                             const float (&acc)[V], float wacc, int cnt,
+                                             bool weighted) {
+    constexpr int D = 32 * V;
+    const float div = weighted ? wacc : static_cast<float>(cnt);
+    const bool upd = cnt > 0 && div > 0.f;
+    const int64_t e0 = row * D + lane * V;
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < V; ++e) {
+        const float v = upd ? acc[e] / div : p.C_prev[e0 + e];
+        p.C_new[e0 + e] = v;
+        if (p.Cx) {
+            const T t = Cvt<T>::from_f(v);
+            static_cast<T *>(p.Cx)[e0 + e] = t;
+            const float f = Cvt<T>::to_f(t);
+            s = fmaf(f, f, s);
+        }
+    }
+    if (p.cn) {
+        s = warp_sum(s);
+        if (lane == 0) p.cn[row] = s;
+    }
+    if (p.wsum && lane == 0) p.wsum[row] = wacc;
+}
+
+template <typename T, int V, bool WEIGHTED>
+__global__ void __launch_bounds__(fz_warps(32 * V * sizeof(T)) * 32, 1)
+    segreduce_final_kernel(const __grid_constant__ CUtensorMap tmX, const FinalParams p) {
+    constexpr unsigned FULL = 0xffffffffu;
+    constexpr int D = 32 * V;
+    constexpr int RB = D * static_cast<int>(sizeof(T));
+    constexpr int NW = fz_warps(RB);
+    constexpr int S = fz_stages(RB);
+    constexpr uint32_t STAGE = FZ_CHUNK * RB;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t bars[NW][S];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t ring = ((raw + 1023u) & ~1023u) + warp * S * STAGE;
+    const uint8_t *ring_g = smem_raw + (ring - raw);
+    const uint32_t bar0 = smem_u32(&bars[warp][0]);
+
+    const int64_t gw = static_cast<int64_t>(blockIdx.x) * NW + warp;
+    if (gw >= static_cast<int64_t>(p.B) * p.rpb) return;
+    const int b = static_cast<int>(gw / p.rpb);
+    const int r = static_cast<int>(gw % p.rpb);
+    const int32_t *offb = p.offsets + static_cast<int64_t>(b) * (p.K + 1);
+    const int p0 = r * p.range;
+    const int p1 = min(offb[p.K], p0 + p.range);
+    if (p0 >= p1) return;
+    const int nchunks = (p1 - p0 + FZ_CHUNK - 1) / FZ_CHUNK;
+    const int32_t *permb = p.perm + static_cast<int64_t>(b) * p.N;
+    const float *wb = WEIGHTED ? p.w + static_cast<int64_t>(b) * p.N : nullptr;
+    const int64_t rowbase = static_cast<int64_t>(b) * p.K;
+    const uint64_t pol = l2_policy_evict_first();
+
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(bar0 + 8u * s, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    // point index of each lane's position in chunk c (-1 past the range)
+    auto load_idx = [&](int c) {
+        const int pos = p0 + FZ_CHUNK * c + lane;
+        return (c < nchunks && pos < p1) ? permb[pos] : -1;
+    };
+    // gathers of chunk c's 32 rows into stage c % S (rows past the range repeat a valid one)
+    auto issue = [&](int c, int idx) {
+        const int first = __shfl_sync(FULL, idx, 0);
+        const int row = b * p.N + (idx >= 0 ? idx : first);
+        const int q1 = __shfl_down_sync(FULL, row, 1);
+        const int q2 = __shfl_down_sync(FULL, row, 2);
+        const int q3 = __shfl_down_sync(FULL, row, 3);
+        const uint32_t bar = bar0 + 8u * (c % S);
+        if (lane == 0) mbar_arrive_expect_tx(bar, STAGE);
+        __syncwarp();
+        if ((lane & 3) == 0)
+            tma_gather4(ring + (c % S) * STAGE + (lane >> 2) * 4 * RB, &tmX, bar, 0, row, q1, q2, q3, pol);
+    };
+
+    // segment holding p0: the largest k with offb[k] <= p0
+    int lo = 0, hi = p.K - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (offb[mid] <= p0) lo = mid; else hi = mid - 1;
+    }
+    int kcur = lo;
+
+    float acc[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) acc[e] = 0.f;
+    float wacc = 0.f;
+    int acck = -1, seg_s = 0, seg_e = 0;
+
+    auto flush = [&]() {
+        const int cnt = seg_e - seg_s;
+        if (seg_s >= p0 && seg_e <= p1) {   // the whole cluster lies in this range
+            finalize_one<T, V>(p, rowbase + acck, lane, acc, wacc, cnt, WEIGHTED);
+            return;
+        }
+        const int side = seg_s < p0 ? 0 : 1;
+        const int64_t slot = (gw * 2 + side);
+        float *sp = p.slots + slot * D + lane * V;
+#pragma unroll
+        for (int e = 0; e < V; ++e) sp[e] = acc[e];
+        if (lane == 0) p.wslots[slot] = wacc;
+        __threadfence();
+        __syncwarp();
+        int old = 0;
+        if (lane == 0) old = atomicAdd(p.arrive + rowbase + acck, 1);
+        old = __shfl_sync(FULL, old, 0);
+        const int r0 = seg_s / p.range, r1 = (seg_e - 1) / p.range;
+        if (old != r1 - r0) return;        // not the last range of this segment to arrive
+        __threadfence();
+        float tot[V];
+#pragma unroll
+        for (int e = 0; e < V; ++e) tot[e] = 0.f;
+        float wt = 0.f;
+        for (int rr = r0; rr <= r1; ++rr) {
+            const int64_t sl = (static_cast<int64_t>(b) * p.rpb + rr) * 2 + (rr == r0 ? 1 : 0);
+            const float *q = p.slots + sl * D + lane * V;
+#pragma unroll
+            for (int e = 0; e < V; ++e) tot[e] += __ldcg(q + e);
+            wt += __ldcg(p.wslots + sl);
+        }
+        finalize_one<T, V>(p, rowbase + acck, lane, tot, wt, cnt, WEIGHTED);
+    };
+
+    // prologue: S - 1 chunks in flight; qi[j] holds the point indices of chunk c + j
+    int qi[S];
+#pragma unroll
+    for (int j = 0; j < S; ++j) qi[j] = load_idx(j);
+#pragma unroll
+    for (int j = 0; j < S - 1; ++j)
+        if (j < nchunks) issue(j, qi[j]);
+    uint32_t phase_bits = 0;   // bit s: parity of the next completion of stage s
+
+    for (int c = 0; c < nchunks; ++c) {
+        const int slot_c = c % S;
+        const int my_i = qi[0];
+        // refill: chunk c + S - 1 goes into the stage chunk c - 1 used (read and fenced below)
+        if (c + S - 1 < nchunks) issue(c + S - 1, qi[S - 1]);
+        float my_w = 1.f;
+        if constexpr (WEIGHTED) my_w = my_i >= 0 ? wb[my_i] : 0.f;
+        const int q = p0 + FZ_CHUNK * c;
+        const int nrows = min(FZ_CHUNK, p1 - q);
+        // clusters of the chunk's positions: segment of pl = kcur + #{j >= 1 : offb[kcur+j] <= pl}
+        const int pl = min(q + lane, p1 - 1);
+        int base = kcur, my_k = -1;
+        while (true) {
+            const int idx = base + 1 + lane;
+            const int o = idx <= p.K ? offb[idx] : INT_MAX;
+            int cnt = 0;
+#pragma unroll
+            for (int stp = 16; stp > 0; stp >>= 1) {
+                const int pr = __shfl_sync(FULL, o, cnt + stp - 1);
+                if (pr <= pl) cnt += stp;
+            }
+            const int o31 = __shfl_sync(FULL, o, 31);
+            if (cnt == 31 && o31 <= pl) cnt = 32;
+            if (my_k < 0 && cnt < 32) my_k = base + cnt;
+            if (!__any_sync(FULL, my_k < 0)) break;
+            base += 32;
+        }
+        kcur = __shfl_sync(FULL, my_k, 31);
+        int prev_k = __shfl_up_sync(FULL, my_k, 1);
+        if (lane == 0) prev_k = acck;
+        const unsigned starts = __ballot_sync(FULL, lane < nrows && my_k != prev_k);
+        // segment bounds of each lane's cluster (read once per run start below)
+        const int my_s = offb[my_k], my_e = offb[my_k + 1];
+        // the next chunk whose gathers will be issued needs its indices
+#pragma unroll
+        for (int j = 0; j + 1 < S; ++j) qi[j] = qi[j + 1];
+        qi[S - 1] = load_idx(c + S);
+
+        if (!mbar_wait_warp(bar0 + 8u * slot_c, (phase_bits >> slot_c) & 1u, nullptr)) {
+            // the wait ran out (recorded in the device error word): let every gather issued so
+            // far land (each wait bounded again) before the CTA's shared memory goes away
+            for (int cc = c; cc < min(nchunks, c + S); ++cc)
+                mbar_wait_warp(bar0 + 8u * (cc % S), static_cast<uint32_t>((cc / S) & 1), nullptr);
+            return;
+        }
+        phase_bits ^= 1u << slot_c;
+        const uint8_t *stage = ring_g + slot_c * STAGE;
+        // run by run: rows [rr, re) belong to one cluster (all warp-uniform)
+        for (int rr = 0; rr < nrows;) {
+            if ((starts >> rr) & 1u) {
+                if (acck >= 0) flush();
+                acck = __shfl_sync(FULL, my_k, rr);
+                seg_s = __shfl_sync(FULL, my_s, rr);
+                seg_e = __shfl_sync(FULL, my_e, rr);
+#pragma unroll
+                for (int e = 0; e < V; ++e) acc[e] = 0.f;
+                wacc = 0.f;
+            }
+            const unsigned later = rr < 31 ? starts & (~0u << (rr + 1)) : 0u;
+            const int re = later ? min(nrows, __ffs(later) - 1) : nrows;
+            if constexpr (WEIGHTED) {
+                for (; rr < re; ++rr) {
+                    const float wv = __shfl_sync(FULL, my_w, rr);
+                    float x[V];
+                    row_vals<T, V>(stage + rr * RB, lane, x);
+#pragma unroll
+                    for (int e = 0; e < V; ++e) acc[e] = fmaf(wv, x[e], acc[e]);
+                    wacc += wv;
+                }
+            } else {
+                wacc += static_cast<float>(re - rr);
+#pragma unroll 4
+                for (; rr < re; ++rr) row_add<T, V>(stage + rr * RB, lane, acc);
+            }
+        }
+        // this stage's reads are done before the engine writes it again
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+    }
+    if (acck >= 0) flush();
+}
+
+// Per batch element (one block): offsets[b, 0..K] and cursor[b, k] as scan_kernel, the arrival
+// counters of segreduce_final_kernel zeroed, and the outputs of every empty cluster written
+// (C_new = C_prev, its rounding, norm and a zero weight sum).
+template <typename T>
+__global__ void __launch_bounds__(SCAN_THREADS)
+    scan_final_kernel(const int32_t *__restrict__ counts, int K, int d, int32_t *__restrict__ offsets,
+                      int32_t *__restrict__ cursor, int32_t *__restrict__ arrive, const float *C_prev,
+                      float *C_new, T *__restrict__ Cx, float *__restrict__ cn, float *__restrict__ wsum) {
+    __shared__ int wtot[SCAN_THREADS / 32];
+    __shared__ int elist[4 * SCAN_THREADS];   // empty clusters of one pass over 4096 counts
+    __shared__ int ecount;
+    const int b = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int32_t *cb = counts + static_cast<int64_t>(b) * K;
+    int32_t *ob = offsets + static_cast<int64_t>(b) * (K + 1);
+    int32_t *cur = cursor + static_cast<int64_t>(b) * K;
+    int32_t *ar = arrive + static_cast<int64_t>(b) * K;
+    int carry = 0;
+    for (int base = 0; base < K; base += 4 * SCAN_THREADS) {
+        const int k0 = base + 4 * tid;
+        int v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = (k0 + e < K) ? cb[k0 + e] : 0;
+        const int tsum = v[0] + v[1] + v[2] + v[3];
+        int incl = tsum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) wtot[wid] = incl;
+        __syncthreads();
+        if (wid == 0) {
+            int x = wtot[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            wtot[lane] = x;
+        }
+        __syncthreads();
+        int ex = carry + incl - tsum + (wid > 0 ? wtot[wid - 1] : 0);
+        unsigned empty = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (k0 + e < K) {
+                ob[k0 + e] = ex;
+                cur[k0 + e] = ex;
+                ar[k0 + e] = 0;
+                if (v[e] == 0) empty |= 1u << e;
+            }
+            ex += v[e];
+        }
+        if (tid == 0) ecount = 0;
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            if ((empty >> e) & 1u) elist[atomicAdd(&ecount, 1)] = k0 + e;
+        __syncthreads();
+        // an empty cluster keeps its centroid: one warp per listed row
+        for (int i = wid; i < ecount; i += SCAN_THREADS / 32) {
+            const int64_t row = static_cast<int64_t>(b) * K + elist[i];
+            float s = 0.f;
+            for (int j = lane; j < d; j += 32) {
+                const float c = C_prev[row * d + j];
+                C_new[row * d + j] = c;
+                if (Cx) {
+                    const T t = Cvt<T>::from_f(c);
+                    Cx[row * d + j] = t;
+                    const float f = Cvt<T>::to_f(t);
+                    s = fmaf(f, f, s);
+                }
+            }
+            if (cn) {
+                s = warp_sum(s);
+                if (lane == 0) cn[row] = s;
+            }
+            if (wsum && lane == 0) wsum[row] = 0.f;
+        }
+        carry += wtot[SCAN_THREADS / 32 - 1];
+        __syncthreads();
+    }
+    if (tid == 0) ob[K] = carry;
+}
+
 }  // namespace upd
 }  // namespace km

@@ -95,7 +95,10 @@ km_status km_prep(const float *C, km_dtype dtype, int64_t B, int64_t K, int64_t 
  *   cn[B,K] fp32 = ||Cx[b,k]||^2, or NULL (then computed into the workspace);
  *   w[B,N] fp32 per-point weights for the inertia, or NULL (all ones);
  *   ids[B,N] int32 out (required); mind[B,N] fp32 out or NULL: the squared distance to the
- *   chosen centroid, max(0, .); inertia[B] fp64 out or NULL: sum_i w_i * mind_i.
+ *   chosen centroid, max(0, .); inertia[B] fp64 out or NULL: sum_i w_i * mind_i;
+ *   counts[B,K] int32 out or NULL: the number of points assigned to each cluster (the
+ *   histogram the Sort-Inverse Update starts from; written by the kernel that writes the ids,
+ *   one atomic per distinct cluster per warp, so the update need not read the ids for it).
  * fp16/bf16 with d % 8 == 0, 8 <= d <= 256 and 16-byte aligned X/Cx run on the tcgen05 tensor
  * cores (fp32 accumulation of <x,c>); every other case runs an exact-fp32 CUDA-core kernel that
  * evaluates sum_j (x_j - c_j)^2 directly. On the tensor-core path mind is formed as
@@ -108,7 +111,8 @@ km_status km_prep(const float *C, km_dtype dtype, int64_t B, int64_t K, int64_t 
  */
 km_status km_assign(const void *X, km_dtype dtype, const void *Cx, const float *cn,
                     const float *w, int64_t B, int64_t N, int64_t K, int64_t d, int32_t *ids,
-                    float *mind, double *inertia, void *ws, size_t ws_bytes, void *stream);
+                    float *mind, double *inertia, int32_t *counts, void *ws, size_t ws_bytes,
+                    void *stream);
 
 /*
  * 1 when km_assign with these arguments runs on the tcgen05 tensor cores, 0 when it runs the
@@ -122,15 +126,33 @@ int km_assign_uses_tensor_cores(km_dtype dtype, int64_t d, const void *X, const 
  *   wsum[b,k]   = sum of w over those points (fp32; NULL allowed)
  *   C_new[b,k]  = sum_i w_i X[b,i,:] / wsum[b,k], or C_prev[b,k] when the cluster is empty.
  * The ids are argsorted per batch by a device counting sort into contiguous per-cluster
- * segments; X is read in sorted order by index (never permuted in memory) and each chunk of
- * sorted positions reduces its runs on chip, merging each run with one vector atomic per
- * coordinate block (technologypulse.uk Flash-KMeans article, "Bottleneck 2"; wispaper blog
- * "2. Sort-Inverse Update"). C_new may alias C_prev. Points whose id lies outside [0,K) are
- * ignored (neither counted nor summed).
+ * segments; X is read in sorted order by index (never permuted in memory) and each range of
+ * sorted positions reduces its runs on chip (technologypulse.uk Flash-KMeans article,
+ * "Bottleneck 2"; wispaper blog "2. Sort-Inverse Update"). For d = 32 * V with rows of 128, 256
+ * or 512 bytes and a 16-byte aligned X, rows are gathered four at a time by the tensor-memory
+ * engine and the divide is fused into the reduction: a run that is a whole cluster is divided
+ * where it was summed, a cluster split over ranges combines its per-range partials in range
+ * order (one merge per segment, no atomics on the sums). Other shapes merge each run into a
+ * sums array with one vector atomic per coordinate block and divide in a second kernel.
+ * C_new may alias C_prev. Points whose id lies outside [0,K) are ignored (neither counted nor
+ * summed). Workspace: km_workspace_size(KM_OP_UPDATE, ...) bytes.
  */
 km_status km_update(const void *X, km_dtype dtype, const int32_t *ids, const float *w, int64_t B,
                     int64_t N, int64_t K, int64_t d, const float *C_prev, float *C_new,
                     int32_t *counts, float *wsum, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * km_update followed by km_prep of the new centroids, in the same pass: besides C_new, counts
+ * and wsum (as km_update) it writes Cx[B,K,d] = C_new rounded to X's dtype and cn[B,K] =
+ * ||Cx||^2 (fp32), the inputs of the next km_assign. This is the update of one Lloyd iteration
+ * as km_fit runs it. Cx and cn are required; C_new may alias C_prev. Same workspace as
+ * km_update. counts_ready != 0 says that counts already holds the histogram of ids (as
+ * km_assign writes it) and the histogram pass is skipped; otherwise counts is written here.
+ */
+km_status km_update_next(const void *X, km_dtype dtype, const int32_t *ids, const float *w,
+                         int64_t B, int64_t N, int64_t K, int64_t d, const float *C_prev,
+                         float *C_new, void *Cx, float *cn, int32_t *counts, int counts_ready,
+                         float *wsum, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * First half of km_update, for callers that combine partial sums across devices (points

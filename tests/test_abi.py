@@ -61,7 +61,7 @@ def test_every_declared_symbol_has_a_typed_binding(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert km.km_abi_version() == 1
+    assert km.km_abi_version() == 2
     assert km.km_status_string(0) == "KM_OK"
     assert km.km_status_string(3) == "KM_ERR_WORKSPACE"
     assert km.km_status_string(99) == "KM_ERR_UNKNOWN"
@@ -107,17 +107,17 @@ def test_argument_errors_return_before_any_launch(lib):
     null = None
     st = P(0)
     # km_assign: null X / Cx / ids
-    assert lib.km_assign(null, 1, fake, null, null, 1, 10, 4, 8, fake, null, null, null, 0, st) == 1
-    assert lib.km_assign(fake, 1, null, null, null, 1, 10, 4, 8, fake, null, null, null, 0, st) == 1
-    assert lib.km_assign(fake, 1, fake, null, null, 1, 10, 4, 8, null, null, null, null, 0, st) == 1
+    assert lib.km_assign(null, 1, fake, null, null, 1, 10, 4, 8, fake, null, null, null, null, 0, st) == 1
+    assert lib.km_assign(fake, 1, null, null, null, 1, 10, 4, 8, fake, null, null, null, null, 0, st) == 1
+    assert lib.km_assign(fake, 1, fake, null, null, 1, 10, 4, 8, null, null, null, null, null, 0, st) == 1
     # bad dtype, bad sizes
-    assert lib.km_assign(fake, 7, fake, null, null, 1, 10, 4, 8, fake, null, null, null, 0, st) == 1
-    assert lib.km_assign(fake, 1, fake, null, null, 0, 10, 4, 8, fake, null, null, null, 0, st) == 1
-    assert lib.km_assign(fake, 1, fake, null, null, 1, 1 << 31, 4, 8, fake, null, null, null, 0, st) == 1
+    assert lib.km_assign(fake, 7, fake, null, null, 1, 10, 4, 8, fake, null, null, null, null, 0, st) == 1
+    assert lib.km_assign(fake, 1, fake, null, null, 0, 10, 4, 8, fake, null, null, null, null, 0, st) == 1
+    assert lib.km_assign(fake, 1, fake, null, null, 1, 1 << 31, 4, 8, fake, null, null, null, null, 0, st) == 1
     # misaligned fp16 pointer
-    assert lib.km_assign(P(0x10001), 1, fake, null, null, 1, 10, 4, 8, fake, null, null, null, 0, st) == 1
+    assert lib.km_assign(P(0x10001), 1, fake, null, null, 1, 10, 4, 8, fake, null, null, null, null, 0, st) == 1
     # tensor-core shape without a workspace
-    assert lib.km_assign(fake, 1, fake, null, null, 1, 10, 4, 128, fake, null, null, null, 0, st) == 3
+    assert lib.km_assign(fake, 1, fake, null, null, 1, 10, 4, 128, fake, null, null, null, null, 0, st) == 3
     # km_update: workspace too small
     assert lib.km_update(fake, 1, fake, null, 1, 10, 4, 8, fake, fake, fake, null, fake, 16, st) == 3
     # km_update_partial: weights without wsum

@@ -92,6 +92,30 @@ def test_assign_matches_oracle(dt, B, N, K, d, weighted, cuda_device):
     check_assign(X, C, ids2)
 
 
+@pytest.mark.parametrize("dt,B,N,K,d", [("f16", 2, 3000, 300, 128), ("bf16", 3, 777, 64, 64),
+                                         ("f32", 1, 4096, 32, 16), ("f16", 1, 129, 1, 128),
+                                         ("f16", 2, 1000, 50, 12), ("f16", 1, 5000, 2, 128)])
+def test_assign_counts_and_the_update_that_reuses_them(dt, B, N, K, d, cuda_device):
+    """km_assign's per-cluster counts equal a histogram of its ids (exact), and the update fed
+    those counts (counts_ready) gives the same centroids as the one that counts for itself."""
+    dtype = DT[dt]
+    X, C = mixture(B, N, d, K, dtype, cuda_device, seed=31 + N + K)
+    Cx, cn = km.km_prep(C, dtype)
+    counts = torch.full((B, K), -7, dtype=torch.int32, device=cuda_device)   # overwritten
+    ids, _, _ = km.km_assign(X, Cx, cn, counts=counts)
+    torch.cuda.synchronize()
+    g = to_np(ids)
+    for b in range(B):
+        np.testing.assert_array_equal(to_np(counts[b]), np.bincount(g[b], minlength=K))
+    Cx1, cn1, Cx2, cn2 = (torch.empty_like(t) for t in (Cx, cn, Cx, cn))
+    C1, c1, _ = km.km_update_next(X, ids, C, Cx1, cn1)
+    C2, c2, _ = km.km_update_next(X, ids, C, Cx2, cn2, counts=counts.clone(), counts_ready=True)
+    torch.cuda.synchronize()
+    assert torch.equal(c1, counts) and torch.equal(c2, counts)
+    torch.testing.assert_close(C2, C1, rtol=1e-5, atol=1e-6)
+    check_update(X, ids, C, C2, c2)
+
+
 def test_tensor_core_distance_precision_bound(cuda_device):
     """Centroids almost on top of their points: the reported distance comes from the expanded
     form ||x||^2 + ||c||^2 - 2<x,c> in fp32, so its absolute error is bounded by a small multiple
@@ -173,6 +197,14 @@ UPD_CASES = [
     ("f32", 2, 600, 17, 1),
     ("f16", 1, 100, 400, 128),       # K > N: empty clusters keep their centroid
     ("f16", 1, 20000, 3, 32),        # few huge segments spanning many warps
+    # the fused reduce-and-divide form (rows of 128, 256, 512 bytes)
+    ("f16", 1, 200000, 3, 128),      # three segments, each split over many ranges
+    ("f32", 2, 3000, 100, 64),
+    ("f32", 1, 5000, 40, 128),
+    ("f16", 1, 3000, 70, 256),
+    ("bf16", 3, 2000, 1, 128),       # K = 1: one segment per problem
+    ("f32", 1, 1000, 10, 32),
+    ("bf16", 40, 700, 30, 64),       # more problems than ranges per problem
 ]
 
 
@@ -194,6 +226,34 @@ def test_update_matches_oracle(dt, B, N, K, d, weighted, cuda_device):
     assert torch.equal(c2, counts)
     torch.testing.assert_close(C2, C_new, rtol=1e-5, atol=1e-6)
     assert torch.equal(Cx2, C2.to(dtype))
+
+
+@pytest.mark.parametrize("dt,B,N,K,d", [("f16", 2, 3000, 300, 128), ("bf16", 1, 50000, 5, 64),
+                                         ("f32", 1, 4000, 33, 16), ("f16", 1, 100, 400, 128)])
+@pytest.mark.parametrize("weighted", [False, True])
+def test_update_next_writes_the_next_assignment_inputs(dt, B, N, K, d, weighted, cuda_device):
+    """km_update_next = km_update plus the rounded centroids and their norms in one pass."""
+    dtype = DT[dt]
+    X, C = mixture(B, N, d, K, dtype, cuda_device, seed=7 + N)
+    w = (torch.rand((B, N), device=cuda_device) * 2 + 0.01) if weighted else None
+    Cx, cn = km.km_prep(C, dtype)
+    ids, _, _ = km.km_assign(X, Cx, cn)
+    C_ref, counts_ref, wsum_ref = km.km_update(X, ids, C, w=w, want_wsum=True)
+    Cx2 = torch.empty_like(Cx)
+    cn2 = torch.empty_like(cn)
+    C_new, counts, wsum = km.km_update_next(X, ids, C, Cx2, cn2, w=w, want_wsum=True)
+    torch.cuda.synchronize()
+    check_update(X, ids, C, C_new, counts, w=w, wsum_gpu=wsum)
+    assert torch.equal(counts, counts_ref)
+    torch.testing.assert_close(C_new, C_ref, rtol=1e-5, atol=1e-6)
+    torch.testing.assert_close(wsum, wsum_ref, rtol=1e-5, atol=1e-6)
+    assert torch.equal(Cx2, C_new.to(dtype))
+    torch.testing.assert_close(cn2.double(), (Cx2.double() ** 2).sum(-1), rtol=2e-6, atol=0)
+    # in place (C_new aliases C_prev), as a fit runs it
+    C_in = C.clone()
+    km.km_update_next(X, ids, C_in, Cx2, cn2, w=w, C_new=C_in)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(C_in, C_ref, rtol=1e-5, atol=1e-6)
 
 
 def test_update_in_place_and_random_ids(cuda_device):
