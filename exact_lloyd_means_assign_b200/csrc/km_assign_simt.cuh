@@ -22,7 +22,7 @@ __global__ void __launch_bounds__(kSimtPts)
     assign_simt_kernel(const T *__restrict__ X, const T *__restrict__ Cx,
                        const float *__restrict__ w, int N, int K, int d, int32_t *__restrict__ ids,
                        float *__restrict__ mind, double *__restrict__ inertia,
-                       int32_t *__restrict__ counts) {
+                       int32_t *__restrict__ counts, int64_t xld) {
     __shared__ float xs[kSimtDC][kSimtPts + 1];
     __shared__ float cs[kSimtKT][kSimtDC];
     __shared__ double red[kSimtPts / 32];
@@ -32,7 +32,7 @@ __global__ void __launch_bounds__(kSimtPts)
     const int64_t i0 = static_cast<int64_t>(blockIdx.x) * kSimtPts;
     const int64_t i = i0 + tid;
     const bool valid = i < N;
-    const T *Xb = X + static_cast<int64_t>(b) * N * d;
+    const T *Xb = X + static_cast<int64_t>(b) * xld * d;   // xld >= N rows per batch element
     const T *Cb = Cx + static_cast<int64_t>(b) * K * d;
 
     float best = INFINITY;
@@ -80,14 +80,10 @@ __global__ void __launch_bounds__(kSimtPts)
         const int64_t gi = static_cast<int64_t>(b) * N + i;
         ids[gi] = bi;
         if (mind) mind[gi] = best;
-        contrib = static_cast<double>(w ? w[gi] : 1.f) * static_cast<double>(best);
+        contrib = static_cast<double>(w ? w[static_cast<int64_t>(b) * xld + i] : 1.f) *
+                  static_cast<double>(best);
     }
-    if (counts) {   // per-cluster point counts, one atomic per distinct cluster in the warp
-        const int key = valid ? bi : -1;
-        const unsigned peers = __match_any_sync(0xffffffffu, key);
-        if (key >= 0 && (tid & 31) == __ffs(peers) - 1)
-            atomicAdd(counts + static_cast<int64_t>(b) * K + key, __popc(peers));
-    }
+    if (counts && valid) atomicAdd(counts + static_cast<int64_t>(b) * K + bi, 1);   // histogram
     if (inertia) {
         contrib = warp_sum(contrib);
         if ((tid & 31) == 0) red[tid >> 5] = contrib;

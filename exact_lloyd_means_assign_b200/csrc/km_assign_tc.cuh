@@ -130,6 +130,7 @@ struct Params {
     int need_dist;  // 1 when the distance / inertia is requested
     uint32_t idesc_main, idesc_aug;
     const float *w;
+    int64_t wld;    // elements between the weights of consecutive batch elements (>= N)
     int32_t *ids;
     float *mind;
     double *inertia;
@@ -636,21 +637,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     if (p.need_dist) {
                         const float md = fmaxf(0.f, 2.f * (best_v + delta));
                         if (p.mind) p.mind[gi] = md;
-                        contrib = static_cast<double>(p.w ? p.w[gi] : 1.f) * static_cast<double>(md);
+                        const float wi = p.w ? p.w[static_cast<int64_t>(b) * p.wld + i] : 1.f;
+                        contrib = static_cast<double>(wi) * static_cast<double>(md);
                     }
                 }
                 if (p.inertia) {
                     contrib = warp_sum(contrib);
                     if (lane == 0) atomicAdd(p.inertia + b, contrib);
                 }
-                if (p.counts) {
-                    // the histogram the update's sort starts from: one atomic per distinct
-                    // cluster among the warp's 32 points
-                    const int key = i < p.N ? best_i : -1;
-                    const unsigned peers = __match_any_sync(0xffffffffu, key);
-                    if (key >= 0 && lane == __ffs(peers) - 1)
-                        atomicAdd(p.counts + static_cast<size_t>(b) * p.K + key, __popc(peers));
-                }
+                // the histogram the update's sort starts from (a reduction without return)
+                if (p.counts && i < p.N) atomicAdd(p.counts + static_cast<size_t>(b) * p.K + best_i, 1);
             }
         }
     }

@@ -289,16 +289,16 @@ km_status finalize_dispatch(const float *sums, const float *wsum, const int32_t 
 template <typename T>
 km_status run_assign_simt(const void *X, const void *Cx, const float *w, int64_t B, int64_t N,
                           int64_t K, int64_t d, int32_t *ids, float *mind, double *inertia,
-                          int32_t *counts, cudaStream_t st) {
+                          int32_t *counts, int64_t xld, cudaStream_t st) {
     const T *Xt = static_cast<const T *>(X);
     const T *Ct = static_cast<const T *>(Cx);
     for (int64_t b0 = 0; b0 < B; b0 += kMaxGridY) {
         const int64_t nb = std::min<int64_t>(kMaxGridY, B - b0);
         dim3 grid(static_cast<unsigned>(ceil_div(N, km::kSimtPts)), static_cast<unsigned>(nb));
         km::assign_simt_kernel<T><<<grid, km::kSimtPts, 0, st>>>(
-            Xt + b0 * N * d, Ct + b0 * K * d, w ? w + b0 * N : nullptr, static_cast<int>(N),
+            Xt + b0 * xld * d, Ct + b0 * K * d, w ? w + b0 * xld : nullptr, static_cast<int>(N),
             static_cast<int>(K), static_cast<int>(d), ids + b0 * N, mind ? mind + b0 * N : nullptr,
-            inertia ? inertia + b0 : nullptr, counts ? counts + b0 * K : nullptr);
+            inertia ? inertia + b0 : nullptr, counts ? counts + b0 * K : nullptr, xld);
         if (launch_status() != KM_OK) return KM_ERR_CUDA;
     }
     return KM_OK;
@@ -364,7 +364,8 @@ km_status launch_assign_tc(const CUtensorMap &tmX, const CUtensorMap &tmC, const
 template <typename T>
 km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float *cn,
                         const float *w, int64_t B, int64_t N, int64_t K, int64_t d, int32_t *ids,
-                        float *mind, double *inertia, int32_t *counts, void *caug, cudaStream_t st) {
+                        float *mind, double *inertia, int32_t *counts, void *caug, int64_t xld,
+                        cudaStream_t st) {
     using namespace km::tc;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return KM_ERR_CUDA;
@@ -383,7 +384,8 @@ km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float 
     {
         const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                                     static_cast<cuuint64_t>(B)};
-        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(N * d * 2)};
+        // batch elements xld rows apart (a mini-batch of each problem is a strided view)
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(xld * d * 2)};
         const cuuint32_t box[3] = {static_cast<cuuint32_t>(KC), static_cast<cuuint32_t>(BM), 1};
         if (enc(&tmX, tdt, 3, const_cast<void *>(X), dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -427,6 +429,7 @@ km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float 
         km::mma_idesc_f16(dt == KM_BF16 ? 1u : 0u, 2 * BM, static_cast<uint32_t>(bn)) | (1u << 13);
     p.idesc_aug = km::mma_idesc_f16(1u, 2 * BM, static_cast<uint32_t>(bn));
     p.w = w;
+    p.wld = xld;
     p.ids = ids;
     p.mind = mind;
     p.inertia = inertia;
@@ -448,10 +451,13 @@ km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float 
 // With accumulate_inertia the objective is added to `inertia` instead of overwriting it (the
 // streamed fit sums it over chunks of points).
 // counts (optional) receive the per-cluster point counts of the assignment (overwritten).
+// X (and w) hold the B batch elements xld >= N rows apart (0: xld = N); ids, mind, counts are
+// compact [B, N] / [B, K].
 km_status do_assign(const void *X, km_dtype dt, const void *Cx, const float *cn, const float *w,
                     int64_t B, int64_t N, int64_t K, int64_t d, int32_t *ids, float *mind,
                     double *inertia, void *caug, cudaStream_t st, bool accumulate_inertia = false,
-                    int32_t *counts = nullptr) {
+                    int32_t *counts = nullptr, int64_t xld = 0) {
+    if (xld == 0) xld = N;
     if (inertia && !accumulate_inertia &&
         cudaMemsetAsync(inertia, 0, static_cast<size_t>(B) * 8, st) != cudaSuccess)
         return KM_ERR_CUDA;
@@ -461,15 +467,16 @@ km_status do_assign(const void *X, km_dtype dt, const void *Cx, const float *cn,
                     B * ceil_div(N, 128) <= kMaxIndex;
     if (tc) {
         if (dt == KM_F16)
-            return run_assign_tc<__half>(X, dt, Cx, cn, w, B, N, K, d, ids, mind, inertia, counts, caug, st);
+            return run_assign_tc<__half>(X, dt, Cx, cn, w, B, N, K, d, ids, mind, inertia, counts, caug,
+                                         xld, st);
         return run_assign_tc<__nv_bfloat16>(X, dt, Cx, cn, w, B, N, K, d, ids, mind, inertia, counts,
-                                            caug, st);
+                                            caug, xld, st);
     }
     switch (dt) {
-        case KM_F32: return run_assign_simt<float>(X, Cx, w, B, N, K, d, ids, mind, inertia, counts, st);
-        case KM_F16: return run_assign_simt<__half>(X, Cx, w, B, N, K, d, ids, mind, inertia, counts, st);
+        case KM_F32: return run_assign_simt<float>(X, Cx, w, B, N, K, d, ids, mind, inertia, counts, xld, st);
+        case KM_F16: return run_assign_simt<__half>(X, Cx, w, B, N, K, d, ids, mind, inertia, counts, xld, st);
         default:
-            return run_assign_simt<__nv_bfloat16>(X, Cx, w, B, N, K, d, ids, mind, inertia, counts, st);
+            return run_assign_simt<__nv_bfloat16>(X, Cx, w, B, N, K, d, ids, mind, inertia, counts, xld, st);
     }
 }
 
@@ -652,13 +659,13 @@ inline bool final_ok(km_dtype dt, const void *X, int64_t B, int64_t N, int64_t d
     return rb == 128 || rb == 256 || rb == 512;
 }
 
-template <typename T, int V, bool WEIGHTED>
+template <typename T, int V, bool WEIGHTED, bool EMA>
 km_status launch_final(const CUtensorMap &tm, km::upd::FinalParams &p, int64_t B, int64_t N,
                        cudaStream_t st) {
     using namespace km::upd;
     constexpr int RB = 32 * V * static_cast<int>(sizeof(T));
     constexpr int NW = fz_warps(RB);
-    if (cudaFuncSetAttribute(segreduce_final_kernel<T, V, WEIGHTED>,
+    if (cudaFuncSetAttribute(segreduce_final_kernel<T, V, WEIGHTED, EMA>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, fz_smem(RB)) != cudaSuccess)
         return KM_ERR_CUDA;
     // one CTA per SM; every warp walks one range of sorted positions of one batch element
@@ -670,7 +677,7 @@ km_status launch_final(const CUtensorMap &tm, km::upd::FinalParams &p, int64_t B
     p.range = static_cast<int>(range);
     p.rpb = static_cast<int>(rpb);
     const int64_t warps = B * rpb;
-    segreduce_final_kernel<T, V, WEIGHTED>
+    segreduce_final_kernel<T, V, WEIGHTED, EMA>
         <<<static_cast<unsigned>(ceil_div(warps, NW)), NW * 32, fz_smem(RB), st>>>(tm, p);
     return launch_status();
 }
@@ -678,8 +685,20 @@ km_status launch_final(const CUtensorMap &tm, km::upd::FinalParams &p, int64_t B
 template <typename T, int V>
 km_status final_weighted(const CUtensorMap &tm, km::upd::FinalParams &p, int64_t B, int64_t N,
                          cudaStream_t st) {
-    return p.w ? launch_final<T, V, true>(tm, p, B, N, st) : launch_final<T, V, false>(tm, p, B, N, st);
+    if (p.Nc)
+        return p.w ? launch_final<T, V, true, true>(tm, p, B, N, st)
+                   : launch_final<T, V, false, true>(tm, p, B, N, st);
+    return p.w ? launch_final<T, V, true, false>(tm, p, B, N, st)
+               : launch_final<T, V, false, false>(tm, p, B, N, st);
 }
+
+// The moving-average form of the fused update (e-means) and the view of a mini-batch: batch
+// element b's points are rows b * xld + x0 + [0, N) of X (and the same offsets into w).
+struct EmaArgs {
+    float alpha;
+    float *Nc, *eS, *eW;
+    int32_t *eCnt;
+};
 
 // One sort-inverse update that writes the new centroids directly (no per-cluster sums array):
 // counts (overwritten), then C_new and, when given, Cx (X's dtype), cn and wsum. Requires
@@ -688,7 +707,9 @@ template <typename T>
 km_status run_update_final(const void *X, km_dtype dt, const int32_t *ids, const float *w,
                            int64_t B, int64_t N, int64_t K, int64_t d, const float *C_prev,
                            float *C_new, void *Cx, float *cn, int32_t *counts, bool have_counts,
-                           float *wsum, void *ws, cudaStream_t st) {
+                           float *wsum, void *ws, cudaStream_t st, int64_t xld = 0, int64_t x0 = 0,
+                           const EmaArgs *ema = nullptr) {
+    if (xld == 0) xld = N;
     using namespace km::upd;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return KM_ERR_CUDA;
@@ -712,7 +733,7 @@ km_status run_update_final(const void *X, km_dtype dt, const int32_t *ids, const
     }
     scan_final_kernel<T><<<static_cast<unsigned>(B), SCAN_THREADS, 0, st>>>(
         counts, static_cast<int>(K), static_cast<int>(d), f.offsets, f.cursor, f.arrive, C_prev,
-        C_new, static_cast<T *>(Cx), cn, wsum);
+        C_new, static_cast<T *>(Cx), cn, wsum, ema ? ema->Nc : nullptr, ema ? ema->alpha : 0.f);
     if (launch_status() != KM_OK) return KM_ERR_CUDA;
     const size_t scatter_smem = smem_bins ? static_cast<size_t>(K + TILE) * 4 : 0;
     for (int64_t b0 = 0; b0 < B; b0 += kMaxGridY) {
@@ -723,12 +744,12 @@ km_status run_update_final(const void *X, km_dtype dt, const int32_t *ids, const
             f.perm + b0 * N, smem_bins);
         if (launch_status() != KM_OK) return KM_ERR_CUDA;
     }
-    // X as [B*N rows, d] with one-row boxes for the four-row gathers
+    // X as [B*xld rows, d] with one-row boxes for the four-row gathers
     CUtensorMap tm;
     const CUtensorMapDataType tdt = dt == KM_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                                     : dt == KM_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                    : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(B * N)};
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(B * xld)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * dtype_size(dt)};
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(d), 1};
     const cuuint32_t estr[2] = {1, 1};
@@ -742,6 +763,8 @@ km_status run_update_final(const void *X, km_dtype dt, const int32_t *ids, const
     p.K = static_cast<int>(K);
     p.range = 0;
     p.rpb = 0;
+    p.xld = static_cast<int>(xld);
+    p.x0 = static_cast<int>(x0);
     p.perm = f.perm;
     p.offsets = f.offsets;
     p.w = w;
@@ -753,6 +776,11 @@ km_status run_update_final(const void *X, km_dtype dt, const int32_t *ids, const
     p.slots = f.slots;
     p.wslots = f.wslots;
     p.arrive = f.arrive;
+    p.alpha = ema ? ema->alpha : 0.f;
+    p.Nc = ema ? ema->Nc : nullptr;
+    p.eS = ema ? ema->eS : nullptr;
+    p.eW = ema ? ema->eW : nullptr;
+    p.eCnt = ema ? ema->eCnt : nullptr;
     constexpr int VV = static_cast<int>(16 / sizeof(T));   // 16-byte rows per lane at most
     const int64_t V = d / 32;
     if (V == VV) return final_weighted<T, VV>(tm, p, B, N, st);
@@ -1082,6 +1110,98 @@ km_status do_emeans(const void *X, km_dtype dt, const float *w, int64_t B, int64
     return KM_OK;
 }
 
+
+// e-means with the fused update (rows of 128, 256 or 512 bytes): the state is (C, Nc) with
+// S = C * Nc, every mini-batch of all B problems is one strided view of X, and per mini-batch
+// there is one assignment (labels, batch counts, the objective added to the epoch's) and one
+// sort-inverse update whose finalize applies the moving average.
+struct EmeansFz {
+    void *Cx;
+    float *cn, *Nc, *eS, *eW, *sizes;
+    int32_t *ids, *eCnt, *bcnt;
+    void *fin;    // the fused update's scratch, then the assignment's (used one after the other)
+};
+inline EmeansFz carve_emeans_fused(Carver &c, int64_t B, int64_t K, int64_t d, km_dtype dt, int64_t batch) {
+    EmeansFz e;
+    const size_t kd = static_cast<size_t>(B * K * d), bk = static_cast<size_t>(B * K);
+    e.Cx = c.take<uint8_t>(kd * dtype_size(dt));
+    e.cn = c.take<float>(bk * 4);
+    e.Nc = c.take<float>(bk * 4);
+    e.eS = c.take<float>(kd * 4);
+    e.eW = c.take<float>(bk * 4);
+    e.sizes = c.take<float>(bk * 4);
+    e.ids = c.take<int32_t>(static_cast<size_t>(B * batch) * 4);
+    e.eCnt = c.take<int32_t>(bk * 4);
+    e.bcnt = c.take<int32_t>(bk * 4);
+    e.fin = c.base ? c.base + c.off : nullptr;
+    Carver f(nullptr);
+    carve_final(f, B, batch, K, d);
+    c.off += std::max(f.off, align_up(ws_assign(B, K, d, dt)));
+    return e;
+}
+
+template <typename T>
+km_status run_emeans_fused(const void *X, km_dtype dt, const float *w, int64_t B, int64_t N,
+                           int64_t K, int64_t d, float *C, int64_t batch, int epochs, float alpha0,
+                           const float *split_u, float eps, double *sse_hist, void *ws,
+                           cudaStream_t st) {
+    Carver c(ws);
+    EmeansFz e = carve_emeans_fused(c, B, K, d, dt, batch);
+    const size_t esz = dtype_size(dt);
+    const int64_t rows = B * K;
+    km::em::fill_f32_kernel<<<static_cast<unsigned>(ceil_div(rows, 256)), 256, 0, st>>>(e.Nc, 1.f, rows);
+    if (launch_status() != KM_OK) return KM_ERR_CUDA;
+    km_status s = prep_dispatch(C, dt, rows, d, e.Cx, e.cn, st);
+    if (s != KM_OK) return s;
+    const int64_t steps = ceil_div(N, batch), T_all = static_cast<int64_t>(epochs) * steps;
+    for (int ep = 0; ep < epochs; ++ep) {
+        const bool last = ep + 1 == epochs;
+        double *sse = sse_hist ? sse_hist + static_cast<int64_t>(ep) * B : nullptr;
+        // the epoch's sums are needed only for the final shift, so only the last epoch keeps them
+        if (cudaMemsetAsync(e.eCnt, 0, static_cast<size_t>(rows) * 4, st) != cudaSuccess ||
+            (w && cudaMemsetAsync(e.eW, 0, static_cast<size_t>(rows) * 4, st) != cudaSuccess) ||
+            (last && cudaMemsetAsync(e.eS, 0, static_cast<size_t>(rows * d) * 4, st) != cudaSuccess) ||
+            (sse && cudaMemsetAsync(sse, 0, static_cast<size_t>(B) * 8, st) != cudaSuccess))
+            return KM_ERR_CUDA;
+        for (int64_t stp = 0; stp < steps; ++stp) {
+            const int64_t n0 = stp * batch, n = std::min(batch, N - n0);
+            const void *Xv = static_cast<const uint8_t *>(X) + static_cast<size_t>(n0 * d) * esz;
+            s = do_assign(Xv, dt, e.Cx, e.cn, w ? w + n0 : nullptr, B, n, K, d, e.ids, nullptr, sse,
+                          e.fin, st, true, e.bcnt, N);
+            if (s != KM_OK) return s;
+            const EmaArgs ea{emeans_alpha(alpha0, static_cast<int64_t>(ep) * steps + stp, T_all), e.Nc,
+                             last ? e.eS : nullptr, w ? e.eW : nullptr, e.eCnt};
+            s = run_update_final<T>(X, dt, e.ids, w, B, n, K, d, C, C, e.Cx, e.cn, e.bcnt, true, nullptr,
+                                    e.fin, st, N, n0, &ea);
+            if (s != KM_OK) return s;
+        }
+        if (split_u && !last) {
+            // sizes = the epoch's point counts (weight sums when weighted)
+            if (w) {
+                if (cudaMemcpyAsync(e.sizes, e.eW, static_cast<size_t>(rows) * 4, cudaMemcpyDeviceToDevice,
+                                    st) != cudaSuccess)
+                    return KM_ERR_CUDA;
+            } else {
+                km::em::i32_to_f32_kernel<<<static_cast<unsigned>(ceil_div(rows, 256)), 256, 0, st>>>(
+                    e.eCnt, e.sizes, rows);
+                if (launch_status() != KM_OK) return KM_ERR_CUDA;
+            }
+            s = run_split(e.sizes, split_u + static_cast<int64_t>(ep) * rows, eps, B, K, d, C, e.Nc,
+                          nullptr, nullptr, st);
+            if (s != KM_OK) return s;
+            s = prep_dispatch(C, dt, rows, d, e.Cx, e.cn, st);
+            if (s != KM_OK) return s;
+        }
+    }
+    if (epochs > 0)
+        return finalize_dispatch(e.eS, w ? e.eW : nullptr, e.eCnt, C, rows, d, C, dt, e.Cx, e.cn, st);
+    return KM_OK;
+}
+
+inline bool emeans_fused_ok(km_dtype dt, const void *X, int64_t B, int64_t N, int64_t d) {
+    return final_ok(dt, X, B, N, d);
+}
+
 }  // namespace
 
 // =================================================================== exported C ABI
@@ -1256,9 +1376,10 @@ size_t km_emeans_workspace_size(int64_t B, int64_t K, int64_t d, km_dtype dtype,
                                 int64_t batch) {
     (void)weighted;   // the weight-sum arrays are always carved
     if (!sizes_ok(B, batch, K, d) || !valid_dtype(dtype)) return 0;
-    Carver c(nullptr);
+    Carver c(nullptr), f(nullptr);
     carve_emeans(c, B, K, d, dtype, batch);
-    return c.off;
+    carve_emeans_fused(f, B, K, d, dtype, batch);
+    return std::max(c.off, f.off);   // covers whichever form runs
 }
 
 km_status km_emeans_fit(const void *X, km_dtype dtype, const float *w, int64_t B, int64_t N,
@@ -1274,6 +1395,19 @@ km_status km_emeans_fit(const void *X, km_dtype dtype, const float *w, int64_t B
     if (!ws || ws_bytes < km_emeans_workspace_size(B, K, d, dtype, w != nullptr, batch) ||
         !aligned(ws, kAlign))
         return KM_ERR_WORKSPACE;
+    if (emeans_fused_ok(dtype, X, B, N, d)) {
+        switch (dtype) {
+            case KM_F32:
+                return run_emeans_fused<float>(X, dtype, w, B, N, K, d, C, batch, epochs, alpha0, split_u,
+                                               split_eps, sse_hist, ws, S(stream));
+            case KM_F16:
+                return run_emeans_fused<__half>(X, dtype, w, B, N, K, d, C, batch, epochs, alpha0, split_u,
+                                                split_eps, sse_hist, ws, S(stream));
+            default:
+                return run_emeans_fused<__nv_bfloat16>(X, dtype, w, B, N, K, d, C, batch, epochs, alpha0,
+                                                       split_u, split_eps, sse_hist, ws, S(stream));
+        }
+    }
     return do_emeans(X, dtype, w, B, N, K, d, C, batch, epochs, alpha0, split_u, split_eps,
                      sse_hist, ws, S(stream));
 }

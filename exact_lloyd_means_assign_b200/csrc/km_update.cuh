@@ -463,8 +463,9 @@ constexpr int FZ_CHUNK = 32;
 
 struct FinalParams {
     int B, N, K, range, rpb;
+    int xld, x0;        // X rows of batch element b: b * xld + x0 + [0, N) (a mini-batch view)
     const int32_t *perm, *offsets;
-    const float *w;
+    const float *w;     // weights of batch element b at w + b * xld + x0
     const float *C_prev;
     float *C_new;
     void *Cx;
@@ -473,6 +474,11 @@ struct FinalParams {
     float *slots;       // [B * rpb * 2, d] partials of split segments
     float *wslots;      // [B * rpb * 2] their weight sums
     int32_t *arrive;    // [B, K] arrival counters, zeroed by scan_final_kernel
+    // moving-average form (e-means): the batch statistics enter the state (C, Nc) instead of
+    // replacing C, and are added to the epoch totals (eS may be null; eW null when unweighted)
+    float alpha;
+    float *Nc, *eS, *eW;
+    int32_t *eCnt;
 };
 
 // warps per CTA and ring depth for a row of RB bytes (one CTA per SM, 192 KB of rings). The
@@ -570,7 +576,43 @@ __device__ __forceinline__ void finalize_one(const FinalParams &p, int64_t row, 
     if (p.wsum && lane == 0) p.wsum[row] = wacc;
 }
 
-template <typename T, int V, bool WEIGHTED>
+// The moving-average step of e-means for cluster row `row` with batch sums s, size n (count,
+// or weight sum) and point count cnt. The state is (C, Nc) with S = C * Nc (the two are equal
+// at the start, after every step and after a split):
+//     Nc' = (1 - a) Nc + a n,   C' = ((1 - a) Nc C + a s) / Nc'   (C kept when Nc' == 0);
+// Cx and cn follow C', and the batch statistics are added to the epoch totals.
+template <typename T, int V>
+__device__ __forceinline__ void finalize_ema(const FinalParams &p, int64_t row, int lane,
+                                             const float (&s)[V], float wacc, int cnt,
+                                             bool weighted) {
+    constexpr int D = 32 * V;
+    const float a = p.alpha, a1 = 1.f - a;
+    const float n = weighted ? wacc : static_cast<float>(cnt);
+    const float nold = p.Nc[row];
+    const float nn = a1 * nold + a * n;
+    const int64_t e0 = row * D + lane * V;
+    float sq = 0.f;
+#pragma unroll
+    for (int e = 0; e < V; ++e) {
+        const float c = p.C_new[e0 + e];
+        const float v = nn > 0.f ? (a1 * nold * c + a * s[e]) / nn : c;
+        p.C_new[e0 + e] = v;
+        const T t = Cvt<T>::from_f(v);
+        static_cast<T *>(p.Cx)[e0 + e] = t;
+        const float f = Cvt<T>::to_f(t);
+        sq = fmaf(f, f, sq);
+        if (p.eS) p.eS[e0 + e] += s[e];
+    }
+    sq = warp_sum(sq);
+    if (lane == 0) {
+        p.cn[row] = sq;
+        p.Nc[row] = nn;
+        p.eCnt[row] += cnt;
+        if (p.eW) p.eW[row] += wacc;
+    }
+}
+
+template <typename T, int V, bool WEIGHTED, bool EMA>
 __global__ void __launch_bounds__(fz_warps(32 * V * sizeof(T)) * 32, 1)
     segreduce_final_kernel(const __grid_constant__ CUtensorMap tmX, const FinalParams p) {
     constexpr unsigned FULL = 0xffffffffu;
@@ -597,7 +639,7 @@ __global__ void __launch_bounds__(fz_warps(32 * V * sizeof(T)) * 32, 1)
     if (p0 >= p1) return;
     const int nchunks = (p1 - p0 + FZ_CHUNK - 1) / FZ_CHUNK;
     const int32_t *permb = p.perm + static_cast<int64_t>(b) * p.N;
-    const float *wb = WEIGHTED ? p.w + static_cast<int64_t>(b) * p.N : nullptr;
+    const float *wb = WEIGHTED ? p.w + static_cast<int64_t>(b) * p.xld + p.x0 : nullptr;
     const int64_t rowbase = static_cast<int64_t>(b) * p.K;
     const uint64_t pol = l2_policy_evict_first();
 
@@ -615,7 +657,7 @@ __global__ void __launch_bounds__(fz_warps(32 * V * sizeof(T)) * 32, 1)
     // gathers of chunk c's 32 rows into stage c % S (rows past the range repeat a valid one)
     auto issue = [&](int c, int idx) {
         const int first = __shfl_sync(FULL, idx, 0);
-        const int row = b * p.N + (idx >= 0 ? idx : first);
+        const int row = b * p.xld + p.x0 + (idx >= 0 ? idx : first);
         const int q1 = __shfl_down_sync(FULL, row, 1);
         const int q2 = __shfl_down_sync(FULL, row, 2);
         const int q3 = __shfl_down_sync(FULL, row, 3);
@@ -643,7 +685,8 @@ __global__ void __launch_bounds__(fz_warps(32 * V * sizeof(T)) * 32, 1)
     auto flush = [&]() {
         const int cnt = seg_e - seg_s;
         if (seg_s >= p0 && seg_e <= p1) {   // the whole cluster lies in this range
-            finalize_one<T, V>(p, rowbase + acck, lane, acc, wacc, cnt, WEIGHTED);
+            if constexpr (EMA) finalize_ema<T, V>(p, rowbase + acck, lane, acc, wacc, cnt, WEIGHTED);
+            else finalize_one<T, V>(p, rowbase + acck, lane, acc, wacc, cnt, WEIGHTED);
             return;
         }
         const int side = seg_s < p0 ? 0 : 1;
@@ -671,7 +714,8 @@ __global__ void __launch_bounds__(fz_warps(32 * V * sizeof(T)) * 32, 1)
             for (int e = 0; e < V; ++e) tot[e] += __ldcg(q + e);
             wt += __ldcg(p.wslots + sl);
         }
-        finalize_one<T, V>(p, rowbase + acck, lane, tot, wt, cnt, WEIGHTED);
+        if constexpr (EMA) finalize_ema<T, V>(p, rowbase + acck, lane, tot, wt, cnt, WEIGHTED);
+        else finalize_one<T, V>(p, rowbase + acck, lane, tot, wt, cnt, WEIGHTED);
     };
 
     // prologue: S - 1 chunks in flight; qi[j] holds the point indices of chunk c + j
@@ -767,12 +811,15 @@ __global__ void __launch_bounds__(fz_warps(32 * V * sizeof(T)) * 32, 1)
 
 // Per batch element (one block): offsets[b, 0..K] and cursor[b, k] as scan_kernel, the arrival
 // counters of segreduce_final_kernel zeroed, and the outputs of every empty cluster written
-// (C_new = C_prev, its rounding, norm and a zero weight sum).
+// (C_new = C_prev, its rounding, norm and a zero weight sum). In the moving-average form (Nc
+// given) a cluster without points in the batch only decays its count, Nc <- (1 - alpha) Nc: its
+// centroid (S / Nc with both decayed) and so Cx and cn stay as they are.
 template <typename T>
 __global__ void __launch_bounds__(SCAN_THREADS)
     scan_final_kernel(const int32_t *__restrict__ counts, int K, int d, int32_t *__restrict__ offsets,
                       int32_t *__restrict__ cursor, int32_t *__restrict__ arrive, const float *C_prev,
-                      float *C_new, T *__restrict__ Cx, float *__restrict__ cn, float *__restrict__ wsum) {
+                      float *C_new, T *__restrict__ Cx, float *__restrict__ cn, float *__restrict__ wsum,
+                      float *__restrict__ Nc, float alpha) {
     __shared__ int wtot[SCAN_THREADS / 32];
     __shared__ int elist[4 * SCAN_THREADS];   // empty clusters of one pass over 4096 counts
     __shared__ int ecount;
@@ -818,6 +865,12 @@ __global__ void __launch_bounds__(SCAN_THREADS)
                 if (v[e] == 0) empty |= 1u << e;
             }
             ex += v[e];
+        }
+        if (Nc) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if ((empty >> e) & 1u) Nc[static_cast<int64_t>(b) * K + k0 + e] *= 1.f - alpha;
+            empty = 0;
         }
         if (tid == 0) ecount = 0;
         __syncthreads();

@@ -50,6 +50,10 @@ def _check_sse(got, ref, X):
     ("f16", 2, 3000, 12, 64, 700, 3, 0.3, False),    # tensor-core assignment, ragged last batch
     ("f32", 1, 2500, 9, 16, 512, 2, 0.5, True),      # exact fp32 assignment, weighted
     ("bf16", 1, 2000, 20, 128, 2000, 2, 0.8, False),  # one mini-batch per epoch
+    # one launch sequence per mini-batch for all problems (fused moving-average update)
+    ("f16", 3, 5000, 40, 128, 1024, 3, 0.4, True),
+    ("f32", 2, 2500, 9, 32, 512, 2, 0.5, True),      # exact fp32 assignment of a strided view
+    ("f16", 4, 1500, 70, 256, 600, 2, 0.6, False),
 ])
 def test_emeans_matches_oracle(dt, B, N, K, d, batch, epochs, alpha0, weighted, cuda_device):
     X, C0 = blobs(B, N, K, d, seed=N + K)
@@ -66,8 +70,9 @@ def test_emeans_matches_oracle(dt, B, N, K, d, batch, epochs, alpha0, weighted, 
     _check_sse(to_np(sse), ref["sse_hist"], X)
 
 
-def test_emeans_zero_epochs_and_alpha_one_full_batch(cuda_device):
-    X, C0 = blobs(1, 1000, 6, 32, seed=3)
+@pytest.mark.parametrize("d", [32, 64])
+def test_emeans_zero_epochs_and_alpha_one_full_batch(d, cuda_device):
+    X, C0 = blobs(1, 1000, 6, d, seed=3)
     X = X.to(torch.float16).to(cuda_device)
     C = C0.to(cuda_device)
     km.km_emeans_fit(X, C, 100, 0, 0.5)
@@ -113,11 +118,12 @@ def test_split_dead_matches_oracle(K, d, cuda_device):
         np.testing.assert_allclose(to_np(Sg)[b][rev], (Cr * Nr[:, None])[rev], rtol=1e-6, atol=1e-7)
 
 
-def test_emeans_split_revives_a_dead_centroid(cuda_device):
+@pytest.mark.parametrize("d", [32, 64])
+def test_emeans_split_revives_a_dead_centroid(d, cuda_device):
     # blob 1 is two sub-blobs at mu1 (1 +/- 0.3 s_k); centroid 3 starts far away and gets no
     # point in the first epoch; its uniform picks blob 1 as donor, and the split with eps = 0.3
     # puts the two halves on the sub-blob centres, so the second epoch separates them cleanly
-    d, eps = 32, 0.3
+    eps = 0.3
     g = torch.Generator().manual_seed(11)
     mu = torch.randn((3, d), generator=g) * 3
     sgn = torch.tensor([1.0 if k % 2 == 0 else -1.0 for k in range(d)])
