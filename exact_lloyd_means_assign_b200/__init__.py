@@ -62,6 +62,8 @@ def _load():
         "km_fit": ([P, I, P, I64, I64, I64, I64, P, I, P, P, P, P, SZ, P], I),
         "km_fit_host": ([P, I, P, I64, I64, I64, I64, P, I, P, P, P, SZ, P], I),
         "km_device_error": ([P, ctypes.POINTER(I)], I),
+        "km_debug_wait_limit": ([ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong)], I),
+        "km_debug_inject": ([I], I),
         "km_assign_uses_tensor_cores": ([I, I64, P, P], I),
         "km_update_noalloc": ([P, I, P, P, I64, I64, I64, I64, P, P, P, P, P], I),
         "km_noalloc_scratch_needed": ([I64, I64, I64, I64], SZ),
@@ -406,3 +408,16 @@ def km_device_error(stream=None):
     if st not in (0, 5):
         raise KMError("km_device_error", st)
     return code.value
+
+
+def km_debug_wait_limit(limit_ns):
+    """Test hook: set the bound of every in-kernel wait (ns); returns the previous bound."""
+    old = ctypes.c_ulonglong(0)
+    _check("km_debug_wait_limit", _load().km_debug_wait_limit(int(limit_ns), ctypes.byref(old)))
+    return old.value
+
+
+def km_debug_inject(mode):
+    """Test hook: 1 = the next tensor-core assignments withhold one point tile (waits run out);
+    0 = off (the default)."""
+    _check("km_debug_inject", _load().km_debug_inject(int(mode)))

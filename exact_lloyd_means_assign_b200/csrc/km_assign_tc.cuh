@@ -426,6 +426,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     } else if (warp == WARP_XPROD) {
         // ------------------------------------------------------------ point tiles and norms
         const uint64_t pol_x = l2_policy_evict_first();
+        // test-only fault switch (off by default): withhold the first point tile of pair 0
+        const bool withhold = blockIdx.x == 0 && *reinterpret_cast<volatile int *>(&g_km_inject) == 1;
         float *dbuf = reinterpret_cast<float *>(sgen + L.delta_off);
         const uint32_t xaug_full_leader0 = map_to_rank(XAUG_FULL(0), 0);
         const uint32_t xaug_full_leader1 = map_to_rank(XAUG_FULL(1), 0);
@@ -438,14 +440,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const int xb = local & 1;
             const uint32_t xph = (local >> 1) & 1;
             if (!mbar_wait_warp(X_EMPTY(xb), xph ^ 1u, abortp)) { ok = false; break; }
-            if (lane == 0) {
+            const bool request = !(withhold && local == 0);
+            if (lane == 0 && request) {
                 mbar_arrive_expect_tx(X_FULL(xb), NKC * XCHUNK);
                 for (int kc = 0; kc < NKC; ++kc)
                     tma_load_3d(sbase + L.x_off + (xb * NKC + kc) * XCHUNK, &tmX, X_FULL(xb),
                                 kc * KC, m0, b, pol_x);
             }
             __syncwarp();
-            ++n_x;
+            if (request) ++n_x;
             // The tile's norms as soon as it lands (this warp has nothing else to do until the
             // next buffer is handed back at the end of the work item before this one).
             if (!mbar_wait_warp(X_FULL(xb), xph, abortp)) { ok = false; break; }

@@ -20,6 +20,12 @@ constexpr unsigned int kDevErrTimeout = 1u;
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s
 constexpr uint32_t kSuspendHintNs = 20000u;                  // per blocking probe
 
+// Limit of every bounded wait (host-settable, for tests that make a wait run out quickly) and a
+// test-only fault switch read by the tensor-core assignment (0 = off, the default; 1 = the first
+// point tile of the first SM pair is never requested, so the waits on it run out).
+__device__ unsigned long long g_km_wait_limit_ns = kWaitLimitNs;
+__device__ int g_km_inject;
+
 // ------------------------------------------------------------------ dtype traits
 
 template <typename T> struct Cvt;
@@ -119,12 +125,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (mbar_test_wait(bar, parity)) return true;
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
+    const unsigned long long limit = *reinterpret_cast<volatile unsigned long long *>(&g_km_wait_limit_ns);
     while (true) {
 #pragma unroll 1
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
         if (abort_flag && *abort_flag) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit) {
             record_dev_error(kDevErrTimeout);
             if (abort_flag) *abort_flag = 1;
             return false;

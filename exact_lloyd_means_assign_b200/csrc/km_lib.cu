@@ -1522,6 +1522,25 @@ km_status km_device_error(void *stream, int *code) {
     return v ? KM_ERR_DEVICE_TIMEOUT : KM_OK;
 }
 
+km_status km_debug_wait_limit(unsigned long long limit_ns, unsigned long long *previous_ns) {
+    if (limit_ns == 0) return KM_ERR_INVALID_ARG;
+    unsigned long long old = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpyFromSymbol(&old, km::g_km_wait_limit_ns, sizeof(old)) != cudaSuccess ||
+        cudaMemcpyToSymbol(km::g_km_wait_limit_ns, &limit_ns, sizeof(limit_ns)) != cudaSuccess)
+        return KM_ERR_CUDA;
+    if (previous_ns) *previous_ns = old;
+    return KM_OK;
+}
+
+km_status km_debug_inject(int mode) {
+    if (mode != 0 && mode != 1) return KM_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpyToSymbol(km::g_km_inject, &mode, sizeof(mode)) != cudaSuccess)
+        return KM_ERR_CUDA;
+    return KM_OK;
+}
+
 }  // extern "C"
 
 // =================================================================== allocation-free update

@@ -245,6 +245,20 @@ km_status km_fit_stream(const void *X_host, km_dtype dtype, const float *w_host,
 km_status km_device_error(void *stream, int *code);
 
 /*
+ * Test hooks for the failure path (no page text has a counterpart). Every wait inside the
+ * kernels is bounded; km_debug_wait_limit sets that bound for the current device (default 4 s;
+ * *previous_ns receives the old value when non-NULL) so a test can make a wait run out quickly.
+ * km_debug_inject(1) makes the next tensor-core assignments withhold the first point tile of the
+ * first SM pair: the waits on it run out, every role of that pair leaves its loop, copies in
+ * flight land, the issued MMAs drain, tensor memory is freed and the kernel returns with bit 0
+ * of the device error word set (km_device_error reports KM_ERR_DEVICE_TIMEOUT); its labels
+ * are left unwritten. km_debug_inject(0) (the default) turns it off. Both synchronise the device
+ * first. No fault, trap or endless loop is involved.
+ */
+km_status km_debug_wait_limit(unsigned long long limit_ns, unsigned long long *previous_ns);
+km_status km_debug_inject(int mode);
+
+/*
  * km_update for callers that cannot allocate device memory: the same computation and outputs
  * as km_update, but the scratch (offsets, cursors, permutation, partial sums) lives in one
  * array of the library itself, KM_NOALLOC_SCRATCH_BYTES (32 MiB) per device. No page text has a
