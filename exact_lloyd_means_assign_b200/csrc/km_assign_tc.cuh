@@ -65,6 +65,8 @@
 // and TMEM is freed.
 #pragma once
 
+#include <utility>
+
 #include "km_common.cuh"
 
 namespace km {
@@ -279,27 +281,37 @@ __device__ __forceinline__ float min3f(float a, float b, float c) {
     return d;
 }
 
-// Minimum packed key over W columns: distance bits with the low log2(W) mantissa bits replaced
-// by the column index (independent chains of eight for ILP).
-template <int W>
-__device__ __forceinline__ float cols_min(const uint32_t (&v)[W]) {
-    constexpr uint32_t MASK = ~static_cast<uint32_t>(W - 1);
-    constexpr int G = W / 8;
-    float m[G];
+// Packed key of column I: the distance bits with the low log2(W) mantissa bits replaced by I.
+// One three-input logic op with the mask held in a register (`mask` = ~(W - 1), kept live by the
+// caller) and I as the immediate; written in PTX so the two constants cannot turn into two ops.
+template <int I>
+__device__ __forceinline__ float pkey(uint32_t v, uint32_t mask) {
+    uint32_t k;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(k) : "r"(v), "r"(mask), "n"(I));   // (v & mask) | I
+    return __uint_as_float(k);
+}
+template <int O, int... E>
+__device__ __forceinline__ float group8_min(const uint32_t *v, uint32_t mask, std::integer_sequence<int, E...>) {
+    const float k[8] = {pkey<O + E>(v[O + E], mask)...};
+    float t = min3f(k[0], k[1], k[2]);
+    t = min3f(t, k[3], k[4]);
+    t = min3f(t, k[5], k[6]);
+    return fminf(t, k[7]);
+}
+template <int W, int... G>
+__device__ __forceinline__ float cols_min_groups(const uint32_t (&v)[W], uint32_t mask,
+                                                 std::integer_sequence<int, G...>) {
+    float m[W / 8] = {group8_min<8 * G>(v, mask, std::make_integer_sequence<int, 8>{})...};
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const int o = 8 * g;
-        auto key = [&](int i) { return __uint_as_float((v[i] & MASK) | static_cast<uint32_t>(i)); };
-        float t = min3f(key(o), key(o + 1), key(o + 2));
-        t = min3f(t, key(o + 3), key(o + 4));
-        t = min3f(t, key(o + 5), key(o + 6));
-        m[g] = fminf(t, key(o + 7));
-    }
+    for (int s = 1; s < W / 8; s *= 2)
 #pragma unroll
-    for (int s = 1; s < G; s *= 2)
-#pragma unroll
-        for (int g = 0; g + s < G; g += 2 * s) m[g] = fminf(m[g], m[g + s]);
+        for (int g = 0; g + s < W / 8; g += 2 * s) m[g] = fminf(m[g], m[g + s]);
     return m[0];
+}
+// Minimum packed key over W columns (independent chains of eight for ILP).
+template <int W>
+__device__ __forceinline__ float cols_min(const uint32_t (&v)[W], uint32_t mask) {
+    return cols_min_groups<W>(v, mask, std::make_integer_sequence<int, W / 8>{});
 }
 
 // NKC = ceil(d / 64): the number of 64-wide chunks of the reduction, fixed per instantiation so
@@ -566,6 +578,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const uint32_t acc_empty_leader0 = map_to_rank(ACC_EMPTY(0), 0);
         const uint32_t acc_empty_leader1 = map_to_rank(ACC_EMPTY(1), 0);
         const uint32_t tlane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + cq * W;
+        uint32_t kmask = ~IMASK;                 // the key mask, held in a register
+        asm volatile("" : "+r"(kmask));
         int abuf = 0;
         uint32_t aph = 0;
         int stage = 0;
@@ -594,7 +608,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster_relaxed(abuf ? acc_empty_leader1 : acc_empty_leader0);
-                const float m = cols_min<W>(v);
+                const float m = cols_min<W>(v, kmask);
                 const uint32_t mb = __float_as_uint(m);
                 const float mv = __uint_as_float(mb & ~IMASK);
                 if (mv < best_v) {

@@ -875,6 +875,7 @@ km_status do_fit(const void *X, km_dtype dt, const float *w, int64_t B, int64_t 
         }
     }
     void *caug = f.rest;  // assignment scratch shares the update region (used one after the other)
+    const bool fused = final_ok(dt, X, B, N, d);
     const size_t cbytes = static_cast<size_t>(B * K * d) * 4;
     km_status s = prep_dispatch(C, dt, B * K, d, f.Cx, f.cn, st);
     if (s != KM_OK) return s;
@@ -883,10 +884,12 @@ km_status do_fit(const void *X, km_dtype dt, const float *w, int64_t B, int64_t 
                                       cudaMemcpyDeviceToDevice, st) != cudaSuccess)
             return KM_ERR_CUDA;
         double *in = inertia_hist ? inertia_hist + static_cast<int64_t>(t) * B : nullptr;
-        s = do_assign(X, dt, f.Cx, f.cn, w, B, N, K, d, f.ids, nullptr, in, caug, st, false, f.counts);
+        // the assignment writes the counts only where the fused update will use them
+        s = do_assign(X, dt, f.Cx, f.cn, w, B, N, K, d, f.ids, nullptr, in, caug, st, false,
+                      fused ? f.counts : nullptr);
         if (s != KM_OK) return s;
         s = do_update(X, dt, f.ids, w, B, N, K, d, C, C, dt, f.Cx, f.cn, f.counts, nullptr, f.rest, st,
-                      true);
+                      fused);
         if (s != KM_OK) return s;
     }
     if (C_hist && cudaMemcpyAsync(C_hist + static_cast<int64_t>(iters) * B * K * d, C, cbytes,
