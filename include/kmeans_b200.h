@@ -71,7 +71,10 @@ int km_abi_version(void);
 /*
  * Bytes of device workspace the entry point `op` needs for these sizes (0 on invalid sizes, and
  * 0 for KM_OP_ASSIGN when the CUDA-core path needs none). `weighted` != 0 when a weight array
- * will be passed and `iters` the iteration count (both matter for KM_OP_FIT_HOST only).
+ * will be passed and `iters` the iteration count. Both matter for KM_OP_FIT_HOST only: that
+ * workspace also holds the device copies of the caller's host buffers, i.e. the weights
+ * (B*N fp32, only when weighted) and the inertia history (iters*B fp64); the other ops keep
+ * those in caller memory, so there they are ignored.
  * The workspace must be 256-byte aligned; its contents need not be initialised.
  */
 size_t km_workspace_size(km_op op, int64_t B, int64_t N, int64_t K, int64_t d, km_dtype dtype,
