@@ -635,7 +635,7 @@ km_status do_update_partial(const void *X, km_dtype dt, const int32_t *ids, cons
         dim3 grid(static_cast<unsigned>(ntiles), static_cast<unsigned>(nb));
         scatter_kernel<<<grid, TILE_THREADS, scatter_smem, st>>>(
             ids + b0 * N, static_cast<int>(N), static_cast<int>(K), u.cursor + b0 * K,
-            u.perm + b0 * N, smem_bins);
+            u.perm + b0 * N, smem_bins, TILE);
         if (launch_status() != KM_OK) return KM_ERR_CUDA;
     }
     km_status s;
@@ -735,13 +735,18 @@ km_status run_update_final(const void *X, km_dtype dt, const int32_t *ids, const
         counts, static_cast<int>(K), static_cast<int>(d), f.offsets, f.cursor, f.arrive, C_prev,
         C_new, static_cast<T *>(Cx), cn, wsum, ema ? ema->Nc : nullptr, ema ? ema->alpha : 0.f);
     if (launch_status() != KM_OK) return KM_ERR_CUDA;
-    const size_t scatter_smem = smem_bins ? static_cast<size_t>(K + TILE) * 4 : 0;
+    // scatter tiles: halved (down to 1024 points) until every SM has at least one block, so a
+    // small problem (an e-means mini-batch) is not sorted by a handful of blocks
+    int64_t stile = TILE;
+    while (stile > 1024 && B * ceil_div(N, stile) < num_sms()) stile /= 2;
+    const int64_t sntiles = ceil_div(N, stile);
+    const size_t scatter_smem = smem_bins ? static_cast<size_t>(K + stile) * 4 : 0;
     for (int64_t b0 = 0; b0 < B; b0 += kMaxGridY) {
         const int64_t nb = std::min<int64_t>(kMaxGridY, B - b0);
-        dim3 grid(static_cast<unsigned>(ntiles), static_cast<unsigned>(nb));
+        dim3 grid(static_cast<unsigned>(sntiles), static_cast<unsigned>(nb));
         scatter_kernel<<<grid, TILE_THREADS, scatter_smem, st>>>(
             ids + b0 * N, static_cast<int>(N), static_cast<int>(K), f.cursor + b0 * K,
-            f.perm + b0 * N, smem_bins);
+            f.perm + b0 * N, smem_bins, static_cast<int>(stile));
         if (launch_status() != KM_OK) return KM_ERR_CUDA;
     }
     // X as [B*xld rows, d] with one-row boxes for the four-row gathers

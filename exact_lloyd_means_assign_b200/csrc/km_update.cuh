@@ -114,13 +114,14 @@ __global__ void __launch_bounds__(SCAN_THREADS)
     if (tid == 0) ob[K] = carry;
 }
 
+// `tile` <= TILE points per block (smaller tiles give small problems more blocks).
 __global__ void __launch_bounds__(TILE_THREADS)
     scatter_kernel(const int32_t *__restrict__ ids, int N, int K, int32_t *__restrict__ cursor,
-                   int32_t *__restrict__ perm, int use_smem) {
+                   int32_t *__restrict__ perm, int use_smem, int tile) {
     extern __shared__ int ssm[];
     const int b = blockIdx.y;
-    const int t0 = blockIdx.x * TILE;
-    const int t1 = min(N, t0 + TILE);
+    const int t0 = blockIdx.x * tile;
+    const int t1 = min(N, t0 + tile);
     const int32_t *idb = ids + static_cast<int64_t>(b) * N;
     int32_t *cur = cursor + static_cast<int64_t>(b) * K;
     int32_t *pb = perm + static_cast<int64_t>(b) * N;
