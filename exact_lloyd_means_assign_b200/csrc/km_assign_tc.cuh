@@ -590,8 +590,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const int xb = local & 1;
             const uint32_t xph = (local >> 1) & 1;
             bool ok = true;
-            float best_v = INFINITY;
-            int best_i = 0;
+            float best_v = INFINITY;   // the best value (key without its column bits) so far
+            uint32_t best_m = 0;       // its packed key
+            int best_j = 0;            // and its tile
             for (int j = 0; j < p.nct; ++j) {
                 if (!mbar_wait_warp(ACC_FULL(abuf), aph, abortp)) { ok = false; break; }
                 tc_fence_after();
@@ -611,14 +612,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 const float m = cols_min<W>(v, kmask);
                 const uint32_t mb = __float_as_uint(m);
                 const float mv = __uint_as_float(mb & ~IMASK);
-                if (mv < best_v) {
+                if (mv < best_v) {   // strict: an earlier tile keeps an equal value
                     best_v = mv;
-                    best_i = j * BN + cq * W + static_cast<int>(mb & IMASK);
+                    best_m = mb;
+                    best_j = j;
                 }
                 abuf ^= 1;
                 if (abuf == 0) aph ^= 1u;
                 if (++stage == S) stage = 0;
             }
+            int best_i = best_j * BN + cq * W + static_cast<int>(best_m & IMASK);
             // Column quarter 0 merges the four quarters of each row and writes the result; the
             // reported distance adds back delta, the rounding of this row's two-piece ||x||^2/2.
             const int slot = local & 1;

@@ -671,7 +671,8 @@ km_status launch_final(const CUtensorMap &tm, km::upd::FinalParams &p, int64_t B
     // one CTA per SM; every warp walks one range of sorted positions of one batch element
     const int64_t total = static_cast<int64_t>(std::min(num_sms(), static_cast<int>(kFinalWarpsMax / NW))) * NW;
     const int64_t rpb0 = std::max<int64_t>(1, total / B);
-    const int64_t range = std::max<int64_t>(64, ceil_div(ceil_div(N, rpb0), 32) * 32);
+    // ranges need not be whole chunks of 32 positions, so every warp gets one
+    const int64_t range = std::max<int64_t>(64, ceil_div(N, rpb0));
     const int64_t rpb = ceil_div(N, range);
     if (rpb > final_rpb_max(B)) return KM_ERR_UNSUPPORTED;   // never: rpb <= rpb0
     p.range = static_cast<int>(range);

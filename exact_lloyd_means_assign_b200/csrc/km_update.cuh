@@ -675,7 +675,12 @@ __global__ void __launch_bounds__(fz_warps(32 * V * sizeof(T)) * 32, 1)
         const int mid = (lo + hi + 1) >> 1;
         if (offb[mid] <= p0) lo = mid; else hi = mid - 1;
     }
-    int kcur = lo;
+    // A window of 32 segment ends kept in registers: lane l holds offb[wbase + 1 + l] (INT_MAX
+    // past K) and wstart = offb[wbase]. Positions only grow, so the window only slides forward
+    // and the per-chunk lookup needs no memory access until a chunk passes its last end.
+    int wbase = lo;
+    int wstart = offb[wbase];
+    int wend = wbase + 1 + lane <= p.K ? offb[wbase + 1 + lane] : INT_MAX;
 
     float acc[V];
 #pragma unroll
@@ -719,10 +724,12 @@ __global__ void __launch_bounds__(fz_warps(32 * V * sizeof(T)) * 32, 1)
         else finalize_one<T, V>(p, rowbase + acck, lane, tot, wt, cnt, WEIGHTED);
     };
 
-    // prologue: S - 1 chunks in flight; qi[j] holds the point indices of chunk c + j
-    int qi[S];
+    // prologue: S - 1 chunks in flight; qi[j] holds the point indices of chunk c + j (loaded
+    // two iterations before their gathers are issued)
+    constexpr int Q = S + 1;
+    int qi[Q];
 #pragma unroll
-    for (int j = 0; j < S; ++j) qi[j] = load_idx(j);
+    for (int j = 0; j < Q; ++j) qi[j] = load_idx(j);
 #pragma unroll
     for (int j = 0; j < S - 1; ++j)
         if (j < nchunks) issue(j, qi[j]);
@@ -737,34 +744,39 @@ __global__ void __launch_bounds__(fz_warps(32 * V * sizeof(T)) * 32, 1)
         if constexpr (WEIGHTED) my_w = my_i >= 0 ? wb[my_i] : 0.f;
         const int q = p0 + FZ_CHUNK * c;
         const int nrows = min(FZ_CHUNK, p1 - q);
-        // clusters of the chunk's positions: segment of pl = kcur + #{j >= 1 : offb[kcur+j] <= pl}
+        // clusters of the chunk's positions: segment of pl = wbase + #{j : offb[wbase+1+j] <= pl},
+        // with the segment bounds [my_s, my_e) taken from the window by shuffles
         const int pl = min(q + lane, p1 - 1);
-        int base = kcur, my_k = -1;
+        int my_k = -1, my_s = 0, my_e = 0;
         while (true) {
-            const int idx = base + 1 + lane;
-            const int o = idx <= p.K ? offb[idx] : INT_MAX;
             int cnt = 0;
 #pragma unroll
             for (int stp = 16; stp > 0; stp >>= 1) {
-                const int pr = __shfl_sync(FULL, o, cnt + stp - 1);
+                const int pr = __shfl_sync(FULL, wend, cnt + stp - 1);
                 if (pr <= pl) cnt += stp;
             }
-            const int o31 = __shfl_sync(FULL, o, 31);
-            if (cnt == 31 && o31 <= pl) cnt = 32;
-            if (my_k < 0 && cnt < 32) my_k = base + cnt;
+            const int w31 = __shfl_sync(FULL, wend, 31);
+            if (cnt == 31 && w31 <= pl) cnt = 32;
+            const int e_here = __shfl_sync(FULL, wend, cnt & 31);
+            const int s_here = __shfl_sync(FULL, wend, (cnt + 31) & 31);
+            if (my_k < 0 && cnt < 32) {
+                my_k = wbase + cnt;
+                my_e = e_here;
+                my_s = cnt == 0 ? wstart : s_here;
+            }
             if (!__any_sync(FULL, my_k < 0)) break;
-            base += 32;
+            // some position lies past the window: slide it by 32 segments
+            wbase += 32;
+            wstart = w31;
+            wend = wbase + 1 + lane <= p.K ? offb[wbase + 1 + lane] : INT_MAX;
         }
-        kcur = __shfl_sync(FULL, my_k, 31);
         int prev_k = __shfl_up_sync(FULL, my_k, 1);
         if (lane == 0) prev_k = acck;
         const unsigned starts = __ballot_sync(FULL, lane < nrows && my_k != prev_k);
-        // segment bounds of each lane's cluster (read once per run start below)
-        const int my_s = offb[my_k], my_e = offb[my_k + 1];
-        // the next chunk whose gathers will be issued needs its indices
+        // the indices of the chunk issued two iterations from now
 #pragma unroll
-        for (int j = 0; j + 1 < S; ++j) qi[j] = qi[j + 1];
-        qi[S - 1] = load_idx(c + S);
+        for (int j = 0; j + 1 < Q; ++j) qi[j] = qi[j + 1];
+        qi[Q - 1] = load_idx(c + Q);
 
         if (!mbar_wait_warp(bar0 + 8u * slot_c, (phase_bits >> slot_c) & 1u, nullptr)) {
             // the wait ran out (recorded in the device error word): let every gather issued so
