@@ -732,23 +732,43 @@ km_status run_update_final(const void *X, km_dtype dt, const int32_t *ids, const
             ids + b0 * N, static_cast<int>(N), static_cast<int>(K), counts + b0 * K, smem_bins);
         if (launch_status() != KM_OK) return KM_ERR_CUDA;
     }
-    scan_final_kernel<T><<<static_cast<unsigned>(B), SCAN_THREADS, 0, st>>>(
-        counts, static_cast<int>(K), static_cast<int>(d), f.offsets, f.cursor, f.arrive, C_prev,
-        C_new, static_cast<T *>(Cx), cn, wsum, ema ? ema->Nc : nullptr, ema ? ema->alpha : 0.f);
-    if (launch_status() != KM_OK) return KM_ERR_CUDA;
     // scatter tiles: halved (down to 1024 points) until every SM has at least one block, so a
     // small problem (an e-means mini-batch) is not sorted by a handful of blocks
     int64_t stile = TILE;
     while (stile > 1024 && B * ceil_div(N, stile) < num_sms()) stile /= 2;
     const int64_t sntiles = ceil_div(N, stile);
-    const size_t scatter_smem = smem_bins ? static_cast<size_t>(K + stile) * 4 : 0;
-    for (int64_t b0 = 0; b0 < B; b0 += kMaxGridY) {
-        const int64_t nb = std::min<int64_t>(kMaxGridY, B - b0);
-        dim3 grid(static_cast<unsigned>(sntiles), static_cast<unsigned>(nb));
-        scatter_kernel<<<grid, TILE_THREADS, scatter_smem, st>>>(
-            ids + b0 * N, static_cast<int>(N), static_cast<int>(K), f.cursor + b0 * K,
-            f.perm + b0 * N, smem_bins, static_cast<int>(stile));
+    if (smem_bins) {
+        // the scan folded into the scatter: slot reservations on a zeroed fill counter
+        const size_t smem = static_cast<size_t>(2 * K + 1 + stile) * 4;
+        if (cudaMemsetAsync(f.cursor, 0, static_cast<size_t>(B * K) * 4, st) != cudaSuccess ||
+            cudaFuncSetAttribute(scatter_final_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (2 * SMEM_K_MAX + 1 + TILE) * 4) != cudaSuccess)
+            return KM_ERR_CUDA;
+        for (int64_t b0 = 0; b0 < B; b0 += kMaxGridY) {
+            const int64_t nb = std::min<int64_t>(kMaxGridY, B - b0);
+            dim3 grid(static_cast<unsigned>(sntiles), static_cast<unsigned>(nb));
+            scatter_final_kernel<T><<<grid, TILE_THREADS, smem, st>>>(
+                ids + b0 * N, counts + b0 * K, static_cast<int>(N), static_cast<int>(K),
+                static_cast<int>(d), static_cast<int>(stile), f.cursor + b0 * K,
+                f.offsets + b0 * (K + 1), f.perm + b0 * N, f.arrive + b0 * K, C_prev + b0 * K * d,
+                C_new + b0 * K * d, Cx ? static_cast<T *>(Cx) + b0 * K * d : nullptr,
+                cn ? cn + b0 * K : nullptr, wsum ? wsum + b0 * K : nullptr,
+                ema ? ema->Nc + b0 * K : nullptr, ema ? ema->alpha : 0.f);
+            if (launch_status() != KM_OK) return KM_ERR_CUDA;
+        }
+    } else {
+        scan_final_kernel<T><<<static_cast<unsigned>(B), SCAN_THREADS, 0, st>>>(
+            counts, static_cast<int>(K), static_cast<int>(d), f.offsets, f.cursor, f.arrive, C_prev,
+            C_new, static_cast<T *>(Cx), cn, wsum, ema ? ema->Nc : nullptr, ema ? ema->alpha : 0.f);
         if (launch_status() != KM_OK) return KM_ERR_CUDA;
+        for (int64_t b0 = 0; b0 < B; b0 += kMaxGridY) {
+            const int64_t nb = std::min<int64_t>(kMaxGridY, B - b0);
+            dim3 grid(static_cast<unsigned>(sntiles), static_cast<unsigned>(nb));
+            scatter_kernel<<<grid, TILE_THREADS, 0, st>>>(
+                ids + b0 * N, static_cast<int>(N), static_cast<int>(K), f.cursor + b0 * K,
+                f.perm + b0 * N, 0, static_cast<int>(stile));
+            if (launch_status() != KM_OK) return KM_ERR_CUDA;
+        }
     }
     // X as [B*xld rows, d] with one-row boxes for the four-row gathers
     CUtensorMap tm;

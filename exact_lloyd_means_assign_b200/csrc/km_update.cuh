@@ -917,5 +917,137 @@ __global__ void __launch_bounds__(SCAN_THREADS)
     if (tid == 0) ob[K] = carry;
 }
 
+// The counting-sort scatter with the scan folded in (K <= SMEM_K_MAX; shared memory: 2K + 1 +
+// tile ints). Every block computes its problem's exclusive offsets of the counts in shared
+// memory, reserves each cluster of its tile a slot range at offs[k] + atomicAdd(fill[b, k],
+// h[k]) (fill zeroed beforehand) and ranks its points into it. The blocks of a problem also
+// share the per-cluster work scan_final_kernel does: tile 0 writes offsets[b, 0..K]; each block
+// zeroes the arrival counters of its share of the clusters and writes the outputs of the empty
+// ones there (C_new = C_prev, Cx, cn, a zero weight sum; in the moving-average form only
+// Nc <- (1 - alpha) Nc).
+template <typename T>
+__global__ void __launch_bounds__(TILE_THREADS)
+    scatter_final_kernel(const int32_t *__restrict__ ids, const int32_t *__restrict__ counts, int N,
+                         int K, int d, int tile, int32_t *__restrict__ fill,
+                         int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
+                         int32_t *__restrict__ arrive, const float *C_prev, float *C_new,
+                         T *__restrict__ Cx, float *__restrict__ cn, float *__restrict__ wsum,
+                         float *__restrict__ Nc, float alpha) {
+    constexpr int NW = TILE_THREADS / 32;
+    extern __shared__ __align__(16) int ssm[];
+    int *offs = ssm;             // [K + 1]: the counts, then their exclusive prefix
+    int *h = ssm + K + 1;        // [K]: the tile's histogram, then its reserved slot cursors
+    int *tids = h + K;           // [tile]: the tile's labels
+    __shared__ int wtot[NW];
+    const int b = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int t0 = blockIdx.x * tile;
+    const int t1 = min(N, t0 + tile);
+    const int64_t kb = static_cast<int64_t>(b) * K;
+    const int32_t *idb = ids + static_cast<int64_t>(b) * N;
+    for (int k = tid; k < K; k += TILE_THREADS) {
+        offs[k] = counts[kb + k];
+        h[k] = 0;
+    }
+    for (int i = t0 + tid; i < t1; i += TILE_THREADS) tids[i - t0] = idb[i];
+    __syncthreads();
+    // exclusive scan in place, 4 * TILE_THREADS counts per pass: thread t takes 4 consecutive
+    // counts with one 16-byte access (a warp reads 512 contiguous bytes: no bank conflicts)
+    int carry = 0;
+    for (int base = 0; base < K; base += 4 * TILE_THREADS) {
+        const int kk = base + 4 * tid;
+        int v[4];
+        if (kk + 3 < K) {
+            const int4 q = *reinterpret_cast<const int4 *>(offs + kk);
+            v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] = kk + e < K ? offs[kk + e] : 0;
+        }
+        const int tsum = v[0] + v[1] + v[2] + v[3];
+        int incl = tsum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) wtot[wid] = incl;
+        __syncthreads();
+        if (wid == 0) {
+            int x = lane < NW ? wtot[lane] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            if (lane < NW) wtot[lane] = x;
+        }
+        __syncthreads();
+        int ex = carry + incl - tsum + (wid > 0 ? wtot[wid - 1] : 0);
+        int o4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            o4[e] = ex;
+            ex += v[e];
+        }
+        if (kk + 3 < K) {
+            *reinterpret_cast<int4 *>(offs + kk) = make_int4(o4[0], o4[1], o4[2], o4[3]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (kk + e < K) offs[kk + e] = o4[e];
+        }
+        carry += wtot[NW - 1];
+        __syncthreads();
+    }
+    if (tid == 0) offs[K] = carry;
+    // the tile's histogram
+    for (int i = tid; i < t1 - t0; i += TILE_THREADS) {
+        const int k = tids[i];
+        if (static_cast<unsigned>(k) < static_cast<unsigned>(K)) atomicAdd(&h[k], 1);
+    }
+    __syncthreads();
+    // this problem's per-cluster work, split over its tiles
+    if (blockIdx.x == 0)
+        for (int k = tid; k <= K; k += TILE_THREADS) offsets[static_cast<int64_t>(b) * (K + 1) + k] = offs[k];
+    const int kb0 = static_cast<int>(static_cast<int64_t>(K) * blockIdx.x / gridDim.x);
+    const int kb1 = static_cast<int>(static_cast<int64_t>(K) * (blockIdx.x + 1) / gridDim.x);
+    for (int k = kb0 + tid; k < kb1; k += TILE_THREADS) {
+        arrive[kb + k] = 0;
+        if (Nc && offs[k + 1] == offs[k]) Nc[kb + k] *= 1.f - alpha;
+    }
+    if (!Nc) {
+        for (int k = kb0 + wid; k < kb1; k += NW) {   // empty clusters keep their centroid
+            if (offs[k + 1] != offs[k]) continue;
+            const int64_t row = kb + k;
+            float s = 0.f;
+            for (int j = lane; j < d; j += 32) {
+                const float c = C_prev[row * d + j];
+                C_new[row * d + j] = c;
+                if (Cx) {
+                    const T t = Cvt<T>::from_f(c);
+                    Cx[row * d + j] = t;
+                    const float f = Cvt<T>::to_f(t);
+                    s = fmaf(f, f, s);
+                }
+            }
+            if (cn) {
+                s = warp_sum(s);
+                if (lane == 0) cn[row] = s;
+            }
+            if (wsum && lane == 0) wsum[row] = 0.f;
+        }
+    }
+    // reserve each cluster of the tile a slot range, then rank the points into it
+    for (int k = tid; k < K; k += TILE_THREADS)
+        if (h[k]) h[k] = offs[k] + atomicAdd(&fill[kb + k], h[k]);
+    __syncthreads();
+    int32_t *pb = perm + static_cast<int64_t>(b) * N;
+    for (int i = tid; i < t1 - t0; i += TILE_THREADS) {
+        const int k = tids[i];
+        if (static_cast<unsigned>(k) < static_cast<unsigned>(K)) pb[atomicAdd(&h[k], 1)] = t0 + i;
+    }
+}
+
 }  // namespace upd
 }  // namespace km
