@@ -12,7 +12,8 @@ larger than the 126 MB L2, so no flush is needed between steps.
 
 A step on the GPU = km_assign (tensor-core FlashAssign; the labels and the per-cluster counts,
 which is all a Lloyd iteration needs: the per-point distance and the inertia are optional
-outputs) + km_update_next (scan, scatter, then the segmented reduce with the division fused in,
+outputs) + km_update_next (scatter with the scan folded in, then the segmented reduce with the
+division fused in,
 writing the new centroids, their rounding and norms for the next assignment): exactly one
 iteration of km_fit's loop without the objective. The assignment with the inertia
 requested is timed separately and reported as "assign_with_inertia_ms".
@@ -64,7 +65,7 @@ def update_bytes(Bw, Nw, Dw, esize):
 
 
 UPDATE_BYTES = update_bytes(B, N, D, 2)
-LAUNCHES_PER_STEP = 5   # caug, assign_tc (+ counts), scan_final, scatter, segreduce_final
+LAUNCHES_PER_STEP = 4   # caug, assign_tc (+ counts), scatter_final (+ scan), segreduce_final
 MIN_TIMED_S = 0.5
 
 
@@ -634,11 +635,11 @@ def run_workload(args):
                                               "mixture's Zipf(1.1) component labels",
                                   "B": Bw, "N": Nw, "K": Kw, "d": Dw, "largest_segment_frac": largest,
                                   "l2": "inputs larger than L2"},
-                          roofline={"bound": "hbm", "kernel": "hist+scan_final+scatter+segreduce_final",
+                          roofline={"bound": "hbm", "kernel": "hist+scatter_final+segreduce_final",
                                     "achieved": ubytes / (u_ms * 1e-3) / 1e9, "peak": peak_bw, "unit": "GB/s",
                                     "frac": ubytes / (u_ms * 1e-3) / 1e9 / peak_bw,
                                     "algorithmic_bytes": ubytes, "peak_source": peak_kind},
-                          gpu_launches=4 * args.steps * blocks,
+                          gpu_launches=3 * args.steps * blocks,
                           cpu_baseline=dict(cpu_desc, value=ubytes / cpu_s / 1e9, unit="GB/s"),
                           clocks=clk.summary(), device_error=km.km_device_error()))
     else:
