@@ -94,7 +94,7 @@ inline UpdateWs carve_update(Carver &c, int64_t B, int64_t N, int64_t K, int64_t
 // slots of split segments (ranges per batch element are at most kFinalWarpsMax / B + 1).
 constexpr int64_t kFinalWarpsMax = 2048;
 struct FinalWs {
-    int32_t *offsets, *cursor, *perm, *arrive;
+    int32_t *offsets, *cursor, *perm, *arrive, *rseg;
     float *slots, *wslots;
 };
 inline int64_t final_rpb_max(int64_t B) { return std::max<int64_t>(1, kFinalWarpsMax / B) + 1; }
@@ -104,6 +104,7 @@ inline FinalWs carve_final(Carver &c, int64_t B, int64_t N, int64_t K, int64_t d
     f.cursor = c.take<int32_t>(static_cast<size_t>(B * K) * 4);
     f.perm = c.take<int32_t>(static_cast<size_t>(B * N) * 4);
     f.arrive = c.take<int32_t>(static_cast<size_t>(B * K) * 4);
+    f.rseg = c.take<int32_t>(static_cast<size_t>(B * final_rpb_max(B)) * 4);
     const int64_t nslots = B * final_rpb_max(B) * 2;
     f.slots = c.take<float>(static_cast<size_t>(nslots * d) * 4);
     f.wslots = c.take<float>(static_cast<size_t>(nslots) * 4);
@@ -659,6 +660,16 @@ inline bool final_ok(km_dtype dt, const void *X, int64_t B, int64_t N, int64_t d
     return rb == 128 || rb == 256 || rb == 512;
 }
 
+// Ranges of sorted positions for the fused reduce: one CTA per SM of `nw` warps, every warp one
+// range of one batch element (ranges need not be whole chunks of 32 positions, so every warp
+// gets one). Returns (range, ranges per batch element).
+inline void final_ranges(int64_t B, int64_t N, int nw, int64_t &range, int64_t &rpb) {
+    const int64_t total = static_cast<int64_t>(std::min(num_sms(), static_cast<int>(kFinalWarpsMax / nw))) * nw;
+    const int64_t rpb0 = std::max<int64_t>(1, total / B);
+    range = std::max<int64_t>(64, ceil_div(N, rpb0));
+    rpb = ceil_div(N, range);   // <= rpb0 < final_rpb_max(B)
+}
+
 template <typename T, int V, bool WEIGHTED, bool EMA>
 km_status launch_final(const CUtensorMap &tm, km::upd::FinalParams &p, int64_t B, int64_t N,
                        cudaStream_t st) {
@@ -668,16 +679,8 @@ km_status launch_final(const CUtensorMap &tm, km::upd::FinalParams &p, int64_t B
     if (cudaFuncSetAttribute(segreduce_final_kernel<T, V, WEIGHTED, EMA>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, fz_smem(RB)) != cudaSuccess)
         return KM_ERR_CUDA;
-    // one CTA per SM; every warp walks one range of sorted positions of one batch element
-    const int64_t total = static_cast<int64_t>(std::min(num_sms(), static_cast<int>(kFinalWarpsMax / NW))) * NW;
-    const int64_t rpb0 = std::max<int64_t>(1, total / B);
-    // ranges need not be whole chunks of 32 positions, so every warp gets one
-    const int64_t range = std::max<int64_t>(64, ceil_div(N, rpb0));
-    const int64_t rpb = ceil_div(N, range);
-    if (rpb > final_rpb_max(B)) return KM_ERR_UNSUPPORTED;   // never: rpb <= rpb0
-    p.range = static_cast<int>(range);
-    p.rpb = static_cast<int>(rpb);
-    const int64_t warps = B * rpb;
+    (void)N;
+    const int64_t warps = B * p.rpb;
     segreduce_final_kernel<T, V, WEIGHTED, EMA>
         <<<static_cast<unsigned>(ceil_div(warps, NW)), NW * 32, fz_smem(RB), st>>>(tm, p);
     return launch_status();
@@ -732,6 +735,10 @@ km_status run_update_final(const void *X, km_dtype dt, const int32_t *ids, const
             ids + b0 * N, static_cast<int>(N), static_cast<int>(K), counts + b0 * K, smem_bins);
         if (launch_status() != KM_OK) return KM_ERR_CUDA;
     }
+    // the reduce's ranges, decided now so the scatter can tabulate where each one starts
+    int64_t range = 0, rpb = 0;
+    final_ranges(B, N, fz_warps(static_cast<int>(d * sizeof(T))), range, rpb);
+    if (rpb > final_rpb_max(B)) return KM_ERR_UNSUPPORTED;   // never (see final_ranges)
     // scatter tiles: halved (down to 1024 points) until every SM has at least one block, so a
     // small problem (an e-means mini-batch) is not sorted by a handful of blocks
     int64_t stile = TILE;
@@ -753,7 +760,8 @@ km_status run_update_final(const void *X, km_dtype dt, const int32_t *ids, const
                 f.offsets + b0 * (K + 1), f.perm + b0 * N, f.arrive + b0 * K, C_prev + b0 * K * d,
                 C_new + b0 * K * d, Cx ? static_cast<T *>(Cx) + b0 * K * d : nullptr,
                 cn ? cn + b0 * K : nullptr, wsum ? wsum + b0 * K : nullptr,
-                ema ? ema->Nc + b0 * K : nullptr, ema ? ema->alpha : 0.f);
+                ema ? ema->Nc + b0 * K : nullptr, ema ? ema->alpha : 0.f, static_cast<int>(range),
+                static_cast<int>(rpb), f.rseg + b0 * rpb);
             if (launch_status() != KM_OK) return KM_ERR_CUDA;
         }
     } else {
@@ -787,8 +795,9 @@ km_status run_update_final(const void *X, km_dtype dt, const int32_t *ids, const
     p.B = static_cast<int>(B);
     p.N = static_cast<int>(N);
     p.K = static_cast<int>(K);
-    p.range = 0;
-    p.rpb = 0;
+    p.range = static_cast<int>(range);
+    p.rpb = static_cast<int>(rpb);
+    p.rseg = smem_bins ? f.rseg : nullptr;
     p.xld = static_cast<int>(xld);
     p.x0 = static_cast<int>(x0);
     p.perm = f.perm;

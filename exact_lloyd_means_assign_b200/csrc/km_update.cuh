@@ -472,6 +472,7 @@ struct FinalParams {
     void *Cx;
     float *cn;
     float *wsum;        // per-cluster weight sums out (counts when unweighted), or null
+    const int32_t *rseg;  // [B * rpb] the segment holding each range's first position, or null
     float *slots;       // [B * rpb * 2, d] partials of split segments
     float *wslots;      // [B * rpb * 2] their weight sums
     int32_t *arrive;    // [B, K] arrival counters, zeroed by scan_final_kernel
@@ -669,11 +670,16 @@ __global__ void __launch_bounds__(fz_warps(32 * V * sizeof(T)) * 32, 1)
             tma_gather4(ring + (c % S) * STAGE + (lane >> 2) * 4 * RB, &tmX, bar, 0, row, q1, q2, q3, pol);
     };
 
-    // segment holding p0: the largest k with offb[k] <= p0
-    int lo = 0, hi = p.K - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (offb[mid] <= p0) lo = mid; else hi = mid - 1;
+    // segment holding p0: the largest k with offb[k] <= p0 (from the scatter's table when given)
+    int lo = 0;
+    if (p.rseg) {
+        lo = p.rseg[gw];
+    } else {
+        int hi = p.K - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (offb[mid] <= p0) lo = mid; else hi = mid - 1;
+        }
     }
     // A window of 32 segment ends kept in registers: lane l holds offb[wbase + 1 + l] (INT_MAX
     // past K) and wstart = offb[wbase]. Positions only grow, so the window only slides forward
@@ -932,7 +938,8 @@ __global__ void __launch_bounds__(TILE_THREADS)
                          int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
                          int32_t *__restrict__ arrive, const float *C_prev, float *C_new,
                          T *__restrict__ Cx, float *__restrict__ cn, float *__restrict__ wsum,
-                         float *__restrict__ Nc, float alpha) {
+                         float *__restrict__ Nc, float alpha, int range, int rpb,
+                         int32_t *__restrict__ rseg) {
     constexpr int NW = TILE_THREADS / 32;
     extern __shared__ __align__(16) int ssm[];
     int *offs = ssm;             // [K + 1]: the counts, then their exclusive prefix
@@ -1008,8 +1015,19 @@ __global__ void __launch_bounds__(TILE_THREADS)
     }
     __syncthreads();
     // this problem's per-cluster work, split over its tiles
-    if (blockIdx.x == 0)
+    if (blockIdx.x == 0) {
         for (int k = tid; k <= K; k += TILE_THREADS) offsets[static_cast<int64_t>(b) * (K + 1) + k] = offs[k];
+        // the segment holding the first position of each range of the reduction that follows
+        for (int r = tid; r < rpb; r += TILE_THREADS) {
+            const int p0 = r * range;
+            int lo = 0, hi = K - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (offs[mid] <= p0) lo = mid; else hi = mid - 1;
+            }
+            rseg[static_cast<int64_t>(b) * rpb + r] = lo;
+        }
+    }
     const int kb0 = static_cast<int>(static_cast<int64_t>(K) * blockIdx.x / gridDim.x);
     const int kb1 = static_cast<int>(static_cast<int64_t>(K) * (blockIdx.x + 1) / gridDim.x);
     for (int k = kb0 + tid; k < kb1; k += TILE_THREADS) {
