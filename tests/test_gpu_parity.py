@@ -205,6 +205,7 @@ UPD_CASES = [
     ("bf16", 3, 2000, 1, 128),       # K = 1: one segment per problem
     ("f32", 1, 1000, 10, 32),
     ("bf16", 40, 700, 30, 64),       # more problems than ranges per problem
+    ("f16", 1, 30000, 20000, 128),   # K above the 16384 shared-memory bins: the two-launch sort
 ]
 
 
