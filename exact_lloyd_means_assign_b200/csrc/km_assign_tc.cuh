@@ -290,28 +290,24 @@ __device__ __forceinline__ float pkey(uint32_t v, uint32_t mask) {
     asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(k) : "r"(v), "r"(mask), "n"(I));   // (v & mask) | I
     return __uint_as_float(k);
 }
-template <int O, int... E>
-__device__ __forceinline__ float group8_min(const uint32_t *v, uint32_t mask, std::integer_sequence<int, E...>) {
-    const float k[8] = {pkey<O + E>(v[O + E], mask)...};
-    float t = min3f(k[0], k[1], k[2]);
-    t = min3f(t, k[3], k[4]);
-    t = min3f(t, k[5], k[6]);
-    return fminf(t, k[7]);
-}
-template <int W, int... G>
-__device__ __forceinline__ float cols_min_groups(const uint32_t (&v)[W], uint32_t mask,
-                                                 std::integer_sequence<int, G...>) {
-    float m[W / 8] = {group8_min<8 * G>(v, mask, std::make_integer_sequence<int, 8>{})...};
+// Minimum of W packed keys and one carried value, as a queue of 3-input mins: W + 1 inputs
+// (odd) take exactly W / 2 operations, and the first W / 6 of them are independent.
+template <int W, int... I>
+__device__ __forceinline__ float keys_min_seq(const uint32_t (&v)[W], uint32_t mask, float carry,
+                                              std::integer_sequence<int, I...>) {
+    static_assert(W % 2 == 0, "an odd number of inputs reduces by 3-input mins alone");
+    float q[2 * W + 1] = {pkey<I>(v[I], mask)..., carry};
+    int head = 0, tail = W + 1;
 #pragma unroll
-    for (int s = 1; s < W / 8; s *= 2)
-#pragma unroll
-        for (int g = 0; g + s < W / 8; g += 2 * s) m[g] = fminf(m[g], m[g + s]);
-    return m[0];
+    for (int s = 0; s < W / 2; ++s) {
+        q[tail++] = min3f(q[head], q[head + 1], q[head + 2]);
+        head += 3;
+    }
+    return q[head];
 }
-// Minimum packed key over W columns (independent chains of eight for ILP).
 template <int W>
-__device__ __forceinline__ float cols_min(const uint32_t (&v)[W], uint32_t mask) {
-    return cols_min_groups<W>(v, mask, std::make_integer_sequence<int, W / 8>{});
+__device__ __forceinline__ float keys_min(const uint32_t (&v)[W], uint32_t mask, float carry) {
+    return keys_min_seq<W>(v, mask, carry, std::make_integer_sequence<int, W>{});
 }
 
 // NKC = ceil(d / 64): the number of 64-wide chunks of the reduction, fixed per instantiation so
@@ -609,14 +605,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster_relaxed(abuf ? acc_empty_leader1 : acc_empty_leader0);
-                const float m = cols_min<W>(v, kmask);
-                const uint32_t mb = __float_as_uint(m);
-                const float mv = __uint_as_float(mb & ~IMASK);
-                if (mv < best_v) {   // strict: an earlier tile keeps an equal value
-                    best_v = mv;
+                // The best value so far (its column bits zero) is one more input of the tree:
+                // it wins every tie with this tile's keys, so the result differs from it only
+                // when a key of this tile is strictly smaller, and an earlier tile keeps an
+                // equal value.
+                const uint32_t mb = __float_as_uint(keys_min<W>(v, kmask, best_v));
+                if (mb != __float_as_uint(best_v)) {
                     best_m = mb;
                     best_j = j;
                 }
+                best_v = __uint_as_float(mb & kmask);
                 abuf ^= 1;
                 if (abuf == 0) aph ^= 1u;
                 if (++stage == S) stage = 0;
