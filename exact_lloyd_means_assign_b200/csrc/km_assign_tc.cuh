@@ -576,48 +576,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const uint32_t tlane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + cq * W;
         uint32_t kmask = ~IMASK;                 // the key mask, held in a register
         asm volatile("" : "+r"(kmask));
+        const bool stage_owner = ew == 0;   // hands the centroid stages back
+        const bool nct_even = (p.nct & 1) == 0;
         int abuf = 0;
         uint32_t aph = 0;
         int stage = 0;
+        // One accumulator tile: wait for its MMAs, load this warp's columns, hand the buffer
+        // back and fold the columns into the running best. `ab` is a constant on the paired path.
+        auto tile = [&](int ab, int j, float &best_v, uint32_t &best_m, int &best_j) -> bool {
+            if (!mbar_wait_warp(ACC_FULL(ab), aph, abortp)) return false;
+            tc_fence_after();
+            // The tile's MMAs are complete: its centroid stage may be refilled.
+            if (stage_owner) {
+                if (lane == 0) mbar_arrive_relaxed(C_EMPTY(stage));
+                if (++stage == S) stage = 0;
+            }
+            __syncwarp();
+            uint32_t v[W];
+            if constexpr (W == 64) tmem_ld_32x32b_x64(tlane + ab * ACC_STRIDE, v);
+            else if constexpr (W == 32) tmem_ld_32x32b_x32(tlane + ab * ACC_STRIDE, v);
+            else tmem_ld_32x32b_x16(tlane + ab * ACC_STRIDE, v);
+            tmem_wait_ld(v);
+            // Every column this warp needs is in registers: hand the accumulator back. The
+            // arrive is relaxed, so it never waits for this warp's output stores.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster_relaxed(ab ? acc_empty_leader1 : acc_empty_leader0);
+            // The best value so far (its column bits zero) is one more input of the tree: it
+            // wins every tie with this tile's keys, so the result differs from it only when a
+            // key of this tile is strictly smaller, and an earlier tile keeps an equal value.
+            const uint32_t mb = __float_as_uint(keys_min<W>(v, kmask, best_v));
+            if (mb != __float_as_uint(best_v)) {
+                best_m = mb;
+                best_j = j;
+            }
+            best_v = __uint_as_float(mb & kmask);
+            return true;
+        };
         int local = 0;
+        int b = t_begin / p.mtiles;          // batch element and pair tile of work item t,
+        int mt = t_begin - b * p.mtiles;     // advanced incrementally
         for (int t = t_begin; t < t_end; ++t, ++local) {
-            const int b = t / p.mtiles;
-            const int m0 = (t % p.mtiles) * (2 * BM) + static_cast<int>(rank) * BM;
+            const int m0 = mt * (2 * BM) + static_cast<int>(rank) * BM;
             const int xb = local & 1;
             const uint32_t xph = (local >> 1) & 1;
             bool ok = true;
             float best_v = INFINITY;   // the best value (key without its column bits) so far
             uint32_t best_m = 0;       // its packed key
             int best_j = 0;            // and its tile
-            for (int j = 0; j < p.nct; ++j) {
-                if (!mbar_wait_warp(ACC_FULL(abuf), aph, abortp)) { ok = false; break; }
-                tc_fence_after();
-                // The tile's MMAs are complete: its centroid stage may be refilled.
-                if (ew == 0 && lane == 0) mbar_arrive_relaxed(C_EMPTY(stage));
-                __syncwarp();
-                uint32_t v[W];
-                if constexpr (W == 64) tmem_ld_32x32b_x64(tlane + abuf * ACC_STRIDE, v);
-                else if constexpr (W == 32) tmem_ld_32x32b_x32(tlane + abuf * ACC_STRIDE, v);
-                else tmem_ld_32x32b_x16(tlane + abuf * ACC_STRIDE, v);
-                tmem_wait_ld(v);
-                // Every column this warp needs is in registers: hand the accumulator back. The
-                // arrive is relaxed, so it never waits for this warp's output stores.
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster_relaxed(abuf ? acc_empty_leader1 : acc_empty_leader0);
-                // The best value so far (its column bits zero) is one more input of the tree:
-                // it wins every tie with this tile's keys, so the result differs from it only
-                // when a key of this tile is strictly smaller, and an earlier tile keeps an
-                // equal value.
-                const uint32_t mb = __float_as_uint(keys_min<W>(v, kmask, best_v));
-                if (mb != __float_as_uint(best_v)) {
-                    best_m = mb;
-                    best_j = j;
+            if (nct_even) {
+                // Tiles come in pairs, buffer 0 then buffer 1, so every item starts on buffer 0.
+                for (int j = 0; j < p.nct; j += 2) {
+                    if (!tile(0, j, best_v, best_m, best_j) || !tile(1, j + 1, best_v, best_m, best_j)) {
+                        ok = false;
+                        break;
+                    }
+                    aph ^= 1u;
                 }
-                best_v = __uint_as_float(mb & kmask);
-                abuf ^= 1;
-                if (abuf == 0) aph ^= 1u;
-                if (++stage == S) stage = 0;
+            } else {
+                for (int j = 0; j < p.nct; ++j) {
+                    if (!tile(abuf, j, best_v, best_m, best_j)) { ok = false; break; }
+                    abuf ^= 1;
+                    if (abuf == 0) aph ^= 1u;
+                }
             }
             int best_i = best_j * BN + cq * W + static_cast<int>(best_m & IMASK);
             // Column quarter 0 merges the four quarters of each row and writes the result; the
@@ -665,6 +686,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 }
                 // the histogram the update's sort starts from (a reduction without return)
                 if (p.counts && i < p.N) atomicAdd(p.counts + static_cast<size_t>(b) * p.K + best_i, 1);
+            }
+            if (++mt == p.mtiles) {
+                mt = 0;
+                ++b;
             }
         }
     }

@@ -60,6 +60,7 @@ TC_CASES = [
     ("f16", 1, 640, 200, 16),
     ("f16", 1, 300, 37, 200),
     ("bf16", 1, 300, 513, 256),
+    ("f16", 2, 2100, 700, 128),     # three 256-wide centroid tiles: an odd count per item
     ("f16", 1, 129, 1, 128),
     ("f16", 2, 100, 300, 24),
     ("bf16", 5, 1, 7, 8),
