@@ -86,9 +86,13 @@ constexpr int NUM_THREADS = 32 * (WARP_EPI0 + NUM_EPI_WARPS);
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_STRIDE = 256;        // TMEM columns between the two accumulators
 constexpr int MAX_STAGES = 8;
+// Slots of the per-row norm roundings (delta): the point buffer is handed back as soon as the
+// item's last accumulator is complete, before the epilogue reads the item's delta, so the
+// producer may run two items ahead of that read.
+constexpr uint32_t DELTA_SLOTS = 4;
 constexpr uint32_t SMEM_LIMIT = 232448;     // 227 KB opt-in per block on sm_100
 constexpr uint32_t SMEM_ATTR = SMEM_LIMIT - 1024;  // dynamic request cap (static smem is tiny)
-constexpr int NUM_BARS_FIXED = 13;
+constexpr int NUM_BARS_FIXED = 15;
 
 // Bytes one CTA stages per centroid tile: nkc chunks of [bn/2 x 64] plus [bn/2 x 16] bf16.
 __host__ __device__ inline uint32_t cstage_bytes(int nkc, int bn) {
@@ -109,7 +113,7 @@ __host__ __device__ inline Layout make_layout(int nkc, int bn, int stages) {
     const uint32_t nbar = NUM_BARS_FIXED + 2 * stages;
     L.slot_off = L.bar_off + nbar * 8u;
     L.delta_off = (L.slot_off + 16u + 15u) & ~15u;
-    L.merge_off = L.delta_off + 2u * BM * 4u;
+    L.merge_off = L.delta_off + DELTA_SLOTS * BM * 4u;
     // per point buffer: three column quarters x 128 rows of (value, index)
     L.total = L.merge_off + 2u * 3u * BM * 8u;
     return L;
@@ -331,10 +335,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     auto X_FULL = [&](int i) { return bar0 + 8u * i; };
     auto X_EMPTY = [&](int i) { return bar0 + 8u * (2 + i); };
     auto XAUG_FULL = [&](int i) { return bar0 + 8u * (4 + i); };
-    auto DELTA_FULL = [&](int i) { return bar0 + 8u * (6 + i); };
-    auto ACC_FULL = [&](int i) { return bar0 + 8u * (8 + i); };
-    auto ACC_EMPTY = [&](int i) { return bar0 + 8u * (10 + i); };
-    const uint32_t DRAIN = bar0 + 8u * 12;
+    auto ACC_FULL = [&](int i) { return bar0 + 8u * (6 + i); };
+    auto ACC_EMPTY = [&](int i) { return bar0 + 8u * (8 + i); };
+    const uint32_t DRAIN = bar0 + 8u * 10;
+    auto DELTA_FULL = [&](int i) { return bar0 + 8u * (11 + i); };   // i < DELTA_SLOTS
     auto C_FULL = [&](int s) { return bar0 + 8u * (NUM_BARS_FIXED + s); };
     auto C_EMPTY = [&](int s) { return bar0 + 8u * (NUM_BARS_FIXED + S + s); };
 
@@ -352,11 +356,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             // item's last accumulator seen complete, so every MMA reading the tile is done)
             mbar_init(X_EMPTY(i), 1 + 4);
             mbar_init(XAUG_FULL(i), 2);      // (leader) point warp of both CTAs
-            mbar_init(DELTA_FULL(i), 1);
             mbar_init(ACC_FULL(i), 1);
             mbar_init(ACC_EMPTY(i), 2 * NUM_EPI_WARPS);       // (leader) epilogue warps of both
         }
         mbar_init(DRAIN, 2);   // one commit per MMA warp
+        for (int i = 0; i < static_cast<int>(DELTA_SLOTS); ++i) mbar_init(DELTA_FULL(i), 1);
         for (int s = 0; s < S; ++s) {
             mbar_init(C_FULL(s), 1);
             mbar_init(C_EMPTY(s), 1);
@@ -460,7 +464,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             // The tile's norms as soon as it lands (this warp has nothing else to do until the
             // next buffer is handed back at the end of the work item before this one).
             if (!mbar_wait_warp(X_FULL(xb), xph, abortp)) { ok = false; break; }
-#pragma unroll 1
+#pragma unroll 2
             for (int rr = 0; rr < BM / 32; ++rr) {
                 const int row = lane + rr * 32;
                 const float half_xn =
@@ -474,7 +478,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 const float tgt = fmaf(half_xn, 0x1p-12f, half_xn);
                 const float x1 = __bfloat162float(__float2bfloat16_rn(tgt));
                 const float x2 = __bfloat162float(__float2bfloat16_rn(tgt - x1));
-                dbuf[xb * BM + row] = (half_xn - x1) - x2;
+                dbuf[(local & (DELTA_SLOTS - 1)) * BM + row] = (half_xn - x1) - x2;
                 // Row of the point-side augmentation in the 32-byte-swizzled layout: the two
                 // 16-byte halves of rows 4..7 of every 8-row group trade places.
                 const uint4 data = make_uint4(pack_bf16x2(x1, x2), pack_bf16x2(1.f, 1.f),
@@ -489,7 +493,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive_cluster(xb ? xaug_full_leader1 : xaug_full_leader0);
-                mbar_arrive(DELTA_FULL(xb));
+                mbar_arrive(DELTA_FULL(local & (DELTA_SLOTS - 1)));
                 mbar_arrive(X_EMPTY(xb));
             }
         }
@@ -583,9 +587,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         int stage = 0;
         // One accumulator tile: wait for its MMAs, load this warp's columns, hand the buffer
         // back and fold the columns into the running best. `ab` is a constant on the paired path.
-        auto tile = [&](int ab, int j, float &best_v, uint32_t &best_m, int &best_j) -> bool {
+        auto tile = [&](int ab, int j, int xb, float &best_v, uint32_t &best_m, int &best_j) -> bool {
             if (!mbar_wait_warp(ACC_FULL(ab), aph, abortp)) return false;
             tc_fence_after();
+            // The item's last tile is complete, so every MMA reading its point tile is done:
+            // the point buffer goes back to the producer now, not after this tile's epilogue.
+            if (cq == 0 && j == p.nct - 1) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(X_EMPTY(xb));
+            }
             // The tile's MMAs are complete: its centroid stage may be refilled.
             if (stage_owner) {
                 if (lane == 0) mbar_arrive_relaxed(C_EMPTY(stage));
@@ -619,7 +629,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         for (int t = t_begin; t < t_end; ++t, ++local) {
             const int m0 = mt * (2 * BM) + static_cast<int>(rank) * BM;
             const int xb = local & 1;
-            const uint32_t xph = (local >> 1) & 1;
             bool ok = true;
             float best_v = INFINITY;   // the best value (key without its column bits) so far
             uint32_t best_m = 0;       // its packed key
@@ -627,7 +636,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             if (nct_even) {
                 // Tiles come in pairs, buffer 0 then buffer 1, so every item starts on buffer 0.
                 for (int j = 0; j < p.nct; j += 2) {
-                    if (!tile(0, j, best_v, best_m, best_j) || !tile(1, j + 1, best_v, best_m, best_j)) {
+                    if (!tile(0, j, xb, best_v, best_m, best_j) || !tile(1, j + 1, xb, best_v, best_m, best_j)) {
                         ok = false;
                         break;
                     }
@@ -635,7 +644,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 }
             } else {
                 for (int j = 0; j < p.nct; ++j) {
-                    if (!tile(abuf, j, best_v, best_m, best_j)) { ok = false; break; }
+                    if (!tile(abuf, j, xb, best_v, best_m, best_j)) { ok = false; break; }
                     abuf ^= 1;
                     if (abuf == 0) aph ^= 1u;
                 }
@@ -649,11 +658,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 midx[(slot * 3 + cq - 1) * BM + row] = best_i;
             }
             float delta = 0.f;
-            if (cq == 0) {
-                if (p.need_dist && ok && mbar_wait_warp(DELTA_FULL(xb), xph, abortp))
-                    delta = dbuf[xb * BM + row];
-                __syncwarp();
-                if (lane == 0) mbar_arrive(X_EMPTY(xb));
+            if (cq == 0 && p.need_dist && ok) {
+                const int ds = local & (DELTA_SLOTS - 1);
+                if (mbar_wait_warp(DELTA_FULL(ds), (local / DELTA_SLOTS) & 1, abortp)) delta = dbuf[ds * BM + row];
             }
             // All four warps of a lane quarter reach this barrier once per work item, then
             // leave together if any of them saw a role give up.
