@@ -92,7 +92,7 @@ constexpr int MAX_STAGES = 8;
 constexpr uint32_t DELTA_SLOTS = 4;
 constexpr uint32_t SMEM_LIMIT = 232448;     // 227 KB opt-in per block on sm_100
 constexpr uint32_t SMEM_ATTR = SMEM_LIMIT - 1024;  // dynamic request cap (static smem is tiny)
-constexpr int NUM_BARS_FIXED = 15;
+constexpr int NUM_BARS_FIXED = 19;
 
 // Bytes one CTA stages per centroid tile: nkc chunks of [bn/2 x 64] plus [bn/2 x 16] bf16.
 __host__ __device__ inline uint32_t cstage_bytes(int nkc, int bn) {
@@ -322,6 +322,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                      const __grid_constant__ CUtensorMap tmA, const Params p) {
     constexpr int W = BN / 4;           // accumulator columns per epilogue warp
     constexpr uint32_t IMASK = W - 1;
+    // Split tiles (bn = 256): each tile's MMAs run as two N = 128 halves with their own
+    // completion and hand-back barriers. Column quarters 0-1 read half 0 while half 1 is still
+    // being computed, so the two warp pairs of a sub-partition work half a tile apart and one
+    // pair's TMEM load overlaps the other pair's compare work. Each CTA supplies 64 centroid rows
+    // per half, so accumulator column c of half h holds centroid (c < 64 ? h * 64 + c :
+    // 128 + h * 64 + c - 64) of the tile: column quarters 0, 1, 2, 3 hold tile columns 0-63,
+    // 128-191, 64-127, 192-255.
+    constexpr bool SPLIT = BN == 256;
     constexpr int CROWS = BN / 2;       // centroid rows each CTA stages per tile
     constexpr uint32_t CCHUNK = CROWS * 128u;   // one [bn/2 x 64] centroid chunk
     extern __shared__ uint8_t smem_raw[];
@@ -335,10 +343,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     auto X_FULL = [&](int i) { return bar0 + 8u * i; };
     auto X_EMPTY = [&](int i) { return bar0 + 8u * (2 + i); };
     auto XAUG_FULL = [&](int i) { return bar0 + 8u * (4 + i); };
+    // accumulator i = 2 * buffer + half (half 1 only with split tiles)
     auto ACC_FULL = [&](int i) { return bar0 + 8u * (6 + i); };
-    auto ACC_EMPTY = [&](int i) { return bar0 + 8u * (8 + i); };
-    const uint32_t DRAIN = bar0 + 8u * 10;
-    auto DELTA_FULL = [&](int i) { return bar0 + 8u * (11 + i); };   // i < DELTA_SLOTS
+    auto ACC_EMPTY = [&](int i) { return bar0 + 8u * (10 + i); };
+    const uint32_t DRAIN = bar0 + 8u * 14;
+    auto DELTA_FULL = [&](int i) { return bar0 + 8u * (15 + i); };   // i < DELTA_SLOTS
     auto C_FULL = [&](int s) { return bar0 + 8u * (NUM_BARS_FIXED + s); };
     auto C_EMPTY = [&](int s) { return bar0 + 8u * (NUM_BARS_FIXED + S + s); };
 
@@ -356,8 +365,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             // item's last accumulator seen complete, so every MMA reading the tile is done)
             mbar_init(X_EMPTY(i), 1 + 4);
             mbar_init(XAUG_FULL(i), 2);      // (leader) point warp of both CTAs
-            mbar_init(ACC_FULL(i), 1);
-            mbar_init(ACC_EMPTY(i), 2 * NUM_EPI_WARPS);       // (leader) epilogue warps of both
+            for (int h = 0; h < 2; ++h) {
+                mbar_init(ACC_FULL(2 * i + h), 1);
+                // (leader) the epilogue warps of both CTAs that read this accumulator (half)
+                mbar_init(ACC_EMPTY(2 * i + h), SPLIT ? NUM_EPI_WARPS : 2 * NUM_EPI_WARPS);
+            }
         }
         mbar_init(DRAIN, 2);   // one commit per MMA warp
         for (int i = 0; i < static_cast<int>(DELTA_SLOTS); ++i) mbar_init(DELTA_FULL(i), 1);
@@ -524,6 +536,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             constexpr uint32_t cchunk16 = CCHUNK >> 4;
             constexpr uint32_t xchunk16 = XCHUNK >> 4;
             const int nk_last = (p.d - (NKC - 1) * KC + 15) / 16;   // K steps of the last chunk
+            // split tiles issue N = BN / 2 per MMA (the N field of the instruction descriptor)
+            constexpr uint32_t NMASK = 0x3Fu << 17;
+            const uint32_t idesc_main = SPLIT ? (p.idesc_main & ~NMASK) | ((BN / 2 >> 3) << 17) : p.idesc_main;
+            const uint32_t idesc_aug = SPLIT ? (p.idesc_aug & ~NMASK) | ((BN / 2 >> 3) << 17) : p.idesc_aug;
             while (t < t_end) {
                 const int xb = local & 1;
                 const uint32_t xph = (local >> 1) & 1;
@@ -535,25 +551,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     if (!mbar_wait_warp(XAUG_FULL(xb), xph, abortp)) break;
                     xaug_local = local;
                 }
-                if (!mbar_wait_warp(ACC_EMPTY(abuf), aph ^ 1u, abortp)) break;
                 if (!mbar_wait_warp(C_FULL(stage), cph, abortp)) break;
-                tc_fence_after();
-                const uint32_t dcol = tmem_base + abuf * ACC_STRIDE;
                 const uint32_t b_lo = cbase_lo + stage * stage16;
                 const uint32_t a_lo = xbase_lo + xb * (NKC * xchunk16);
-                if (issuer) {
+                bool fail = false;
 #pragma unroll
-                    for (int kc = 0; kc < NKC; ++kc)
+                for (int h = 0; h < (SPLIT ? 2 : 1); ++h) {
+                    if (!mbar_wait_warp(ACC_EMPTY(2 * abuf + h), aph ^ 1u, abortp)) { fail = true; break; }
+                    tc_fence_after();
+                    // half h: accumulator columns h * 128.., centroid rows h * 64.. of each CTA
+                    const uint32_t dcol = tmem_base + abuf * ACC_STRIDE + h * (BN / 2);
+                    const uint32_t bm_lo = b_lo + h * ((BN / 4) * 128u >> 4);
+                    const uint32_t ba_lo = b_lo + NKC * cchunk16 + h * ((BN / 4) * 32u >> 4);
+                    if (issuer) {
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            if (kc + 1 < NKC || kk < nk_last)
-                                tc_mma_pair(dcol, a_lo + kc * xchunk16 + kk * 2, DESC_HI_SW128,
-                                            b_lo + kc * cchunk16 + kk * 2, DESC_HI_SW128,
-                                            p.idesc_main, (kc | kk) != 0 ? 1u : 0u);
-                    tc_mma_pair(dcol, xaug_lo + xb * (XAUG_BYTES >> 4), DESC_HI_SW32,
-                                b_lo + NKC * cchunk16, DESC_HI_SW32, p.idesc_aug, 1u);
-                    tc_commit_pair_both(ACC_FULL(abuf));
+                        for (int kc = 0; kc < NKC; ++kc)
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                if (kc + 1 < NKC || kk < nk_last)
+                                    tc_mma_pair(dcol, a_lo + kc * xchunk16 + kk * 2, DESC_HI_SW128,
+                                                bm_lo + kc * cchunk16 + kk * 2, DESC_HI_SW128,
+                                                idesc_main, (kc | kk) != 0 ? 1u : 0u);
+                        tc_mma_pair(dcol, xaug_lo + xb * (XAUG_BYTES >> 4), DESC_HI_SW32,
+                                    ba_lo, DESC_HI_SW32, idesc_aug, 1u);
+                        tc_commit_pair_both(ACC_FULL(2 * abuf + h));
+                    }
+                    __syncwarp();
                 }
+                if (fail) break;
                 __syncwarp();
                 aph ^= 1u;
                 g += 2;
@@ -575,12 +600,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const float *dbuf = reinterpret_cast<const float *>(sgen + L.delta_off);
         float *mval = reinterpret_cast<float *>(sgen + L.merge_off);
         int *midx = reinterpret_cast<int *>(sgen + L.merge_off + 2u * 3u * BM * 4u);
-        const uint32_t acc_empty_leader0 = map_to_rank(ACC_EMPTY(0), 0);
-        const uint32_t acc_empty_leader1 = map_to_rank(ACC_EMPTY(1), 0);
+        const int half = SPLIT ? cq >> 1 : 0;   // the accumulator half this warp reads
+        const uint32_t acc_empty_leader0 = map_to_rank(ACC_EMPTY(half), 0);
+        const uint32_t acc_empty_leader1 = map_to_rank(ACC_EMPTY(2 + half), 0);
         const uint32_t tlane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + cq * W;
+        // first tile column of this warp's accumulator columns
+        const int cbase = SPLIT ? (cq & 1) * 128 + (cq >> 1) * 64 : cq * W;
         uint32_t kmask = ~IMASK;                 // the key mask, held in a register
         asm volatile("" : "+r"(kmask));
-        const bool stage_owner = ew == 0;   // hands the centroid stages back
+        // Whole-tile completions are seen by warps of the last half: the last one hands the
+        // centroid stages back, and column quarter 2 (0 without split tiles) the point buffer.
+        const int last_cq = SPLIT ? 2 : 0;
+        const bool stage_owner = ew == (SPLIT ? 8 : 0);
         const bool nct_even = (p.nct & 1) == 0;
         int abuf = 0;
         uint32_t aph = 0;
@@ -588,11 +619,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         // One accumulator tile: wait for its MMAs, load this warp's columns, hand the buffer
         // back and fold the columns into the running best. `ab` is a constant on the paired path.
         auto tile = [&](int ab, int j, int xb, float &best_v, uint32_t &best_m, int &best_j) -> bool {
-            if (!mbar_wait_warp(ACC_FULL(ab), aph, abortp)) return false;
+            if (!mbar_wait_warp(ACC_FULL(2 * ab + half), aph, abortp)) return false;
             tc_fence_after();
             // The item's last tile is complete, so every MMA reading its point tile is done:
             // the point buffer goes back to the producer now, not after this tile's epilogue.
-            if (cq == 0 && j == p.nct - 1) {
+            if (cq == last_cq && j == p.nct - 1) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(X_EMPTY(xb));
             }
@@ -649,7 +680,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     if (abuf == 0) aph ^= 1u;
                 }
             }
-            int best_i = best_j * BN + cq * W + static_cast<int>(best_m & IMASK);
+            int best_i = best_j * BN + cbase + static_cast<int>(best_m & IMASK);
             // Column quarter 0 merges the four quarters of each row and writes the result; the
             // reported distance adds back delta, the rounding of this row's two-piece ||x||^2/2.
             const int slot = local & 1;
@@ -668,9 +699,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             if (cq == 0) {
 #pragma unroll
                 for (int o = 0; o < 3; ++o) {
+                    // a quarter's best may come from any tile: equal values keep the lower index
                     const float ob = mval[(slot * 3 + o) * BM + row];
                     const int oi = midx[(slot * 3 + o) * BM + row];
-                    if (ob < best_v) {   // quarters come in column order: ties keep the lower
+                    if (ob < best_v || (ob == best_v && oi < best_i)) {
                         best_v = ob;
                         best_i = oi;
                     }
