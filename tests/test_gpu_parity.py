@@ -144,6 +144,33 @@ def test_duplicate_centroids_go_to_lowest_index(dt, d, cuda_device):
     np.testing.assert_array_equal(g[ids_ref == 3], 3)
 
 
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_duplicates_in_later_tiles_and_earlier_column_quarters(dt, cuda_device):
+    """K = 1024 in 256-column tiles: each copy below sits in a later tile than its original and
+    in a column quarter that the per-row merge visits first (or in another half of the split
+    tile), so the lowest index must win on the (value, index) order, not on the visiting order."""
+    dtype = DT[dt]
+    X, C = mixture(1, 4000, 128, 1024, dtype, cuda_device, seed=11)
+    g = torch.Generator().manual_seed(12)
+    pairs = [(100, 300), (140, 260), (70, 600), (200, 1000), (5, 900)]
+    rows = []
+    for lo, hi in pairs:
+        C[0, hi] = C[0, lo]
+        near = C[0, lo].cpu() + 0.01 * torch.randn((100, 128), generator=g)
+        rows.append(near)
+    X[0, :500] = torch.cat(rows).to(dtype).to(cuda_device)
+    Cx, cn = km.km_prep(C, dtype)
+    ids, _, _ = km.km_assign(X, Cx, cn)
+    torch.cuda.synchronize()
+    got = to_np(ids)[0]
+    ids_ref, _, _, _ = oracle.assign(oracle.as_f64(X.cpu()), oracle.round_to_dtype(C.cpu(), dtype))
+    ref = ids_ref[0]
+    for lo, hi in pairs:
+        assert not (got == hi).any()
+        np.testing.assert_array_equal(got[ref == lo], lo)
+    assert sum((ref == lo).sum() for lo, _ in pairs) >= 400
+
+
 @pytest.mark.parametrize("dt,d,K", [("f16", 128, 300), ("bf16", 128, 300), ("f16", 64, 100),
                                      ("f16", 256, 60), ("bf16", 8, 300), ("f32", 16, 300)])
 def test_points_on_duplicate_centroids_take_lowest_index(dt, d, K, cuda_device):
