@@ -357,14 +357,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const bool leader = rank == 0;
     volatile int *abortp = &abort_flag;
 
+    // Warps computing the point tiles' norms: the point warp, joined in resident mode by the
+    // centroid warp (which then only hands stages back), so the work is spread over two
+    // sub-partitions instead of loading one.
+    const int nnorm = p.resident ? 2 : 1;
+    // Rows [r0, r1) of point buffer xb (work item `local`): ||x||^2/2 split into two bf16 pieces
+    // for the point side of the norm step, and delta, the rounding left over.
+    auto norm_rows = [&](int xb, int local, int r0, int r1) {
+        float *dbuf = reinterpret_cast<float *>(sgen + L.delta_off);
+        const int lane = threadIdx.x & 31;
+#pragma unroll 2
+        for (int row = r0 + lane; row < r1; row += 32) {
+            const float half_xn =
+                0.5f * tile_row_sqnorm<T>(sgen + L.x_off + xb * NKC * XCHUNK, NKC, row);
+            // The split carries ||x||^2/2 raised by 2^-12 of itself. The accumulator is then
+            // d/2 + (about 2^-13 ||x||^2), positive even for a point on its centroid, since the
+            // two-piece split (2^-18 relative) and the fp32 reduction (below 2^-15 ||x||^2) err
+            // by less. Keys of positive floats order ties by index the way the min expects
+            // (lowest index wins); delta takes the raise back out of the reported distance, and
+            // a constant per row cannot change the argmin.
+            const float tgt = fmaf(half_xn, 0x1p-12f, half_xn);
+            const float x1 = __bfloat162float(__float2bfloat16_rn(tgt));
+            const float x2 = __bfloat162float(__float2bfloat16_rn(tgt - x1));
+            dbuf[(local & (DELTA_SLOTS - 1)) * BM + row] = (half_xn - x1) - x2;
+            // Row of the point-side augmentation in the 32-byte-swizzled layout: the two
+            // 16-byte halves of rows 4..7 of every 8-row group trade places.
+            const uint4 data = make_uint4(pack_bf16x2(x1, x2), pack_bf16x2(1.f, 1.f),
+                                          pack_bf16x2(1.f, 0.f), 0u);
+            const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+            uint8_t *rp = sgen + L.xaug_off + xb * XAUG_BYTES + row * 32;
+            const int sw = (row >> 2) & 1;
+            *reinterpret_cast<uint4 *>(rp + 16 * sw) = data;
+            *reinterpret_cast<uint4 *>(rp + 16 * (1 - sw)) = zero;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+    };
     if (threadIdx.x == 0) {
         abort_flag = 0;
         for (int i = 0; i < 2; ++i) {
             mbar_init(X_FULL(i), 1);
             // own point warp (done reading the tile) + own column-quarter-0 epilogue warps (the
             // item's last accumulator seen complete, so every MMA reading the tile is done)
-            mbar_init(X_EMPTY(i), 1 + 4);
-            mbar_init(XAUG_FULL(i), 2);      // (leader) point warp of both CTAs
+            mbar_init(X_EMPTY(i), nnorm + 4);
+            mbar_init(XAUG_FULL(i), 2 * nnorm);   // (leader) the norm warps of both CTAs
             for (int h = 0; h < 2; ++h) {
                 mbar_init(ACC_FULL(2 * i + h), 1);
                 // (leader) the epilogue warps of both CTAs that read this accumulator (half)
@@ -372,7 +408,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             }
         }
         mbar_init(DRAIN, 2);   // one commit per MMA warp
-        for (int i = 0; i < static_cast<int>(DELTA_SLOTS); ++i) mbar_init(DELTA_FULL(i), 1);
+        for (int i = 0; i < static_cast<int>(DELTA_SLOTS); ++i) mbar_init(DELTA_FULL(i), nnorm);
         for (int s = 0; s < S; ++s) {
             mbar_init(C_FULL(s), 1);
             mbar_init(C_EMPTY(s), 1);
@@ -404,46 +440,60 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 
     if (warp == WARP_CPROD) {
         // ------------------------------------------------------------ centroid producer
-        if (lane == 0) {
-            const uint64_t pol_c = l2_policy_evict_last();
-            int stage = 0;
-            uint32_t cph = 0;
-            long long n_c = 0;
-            bool ok = true;
-            int cur_b = -1;   // batch element whose centroid tiles the ring holds (resident mode)
-            for (int t = t_begin; t < t_end && ok; ++t) {
-                const int b = t / p.mtiles;
-                // Resident mode (the ring holds every tile of a batch element: stage j = tile j):
-                // the tiles are loaded again only when the batch element changes; otherwise the
-                // stage's phase just advances.
-                const bool reload = !p.resident || b != cur_b;
-                cur_b = b;
-                for (int j = 0; j < p.nct; ++j) {
-                    const int crow = j * BN + static_cast<int>(rank) * CROWS;
-                    if (!mbar_wait(C_EMPTY(stage), cph ^ 1u, abortp)) { ok = false; break; }
-                    if (!reload) {
-                        if (leader) mbar_arrive(C_FULL(stage));
-                        ++n_c;
-                        if (++stage == S) { stage = 0; cph ^= 1u; }
-                        continue;
-                    }
-                    if (leader) mbar_arrive_expect_tx(C_FULL(stage), stage_tx);
-                    const uint32_t sdst = sbase + L.c_off + stage * L.stage;
-                    const uint32_t lbar = map_to_rank(C_FULL(stage), 0);
-                    for (int kc = 0; kc < NKC; ++kc)
-                        tma_load_3d_pair(sdst + kc * CCHUNK, &tmC, lbar, kc * KC, crow, b, pol_c);
-                    tma_load_3d_pair(sdst + NKC * CCHUNK, &tmA, lbar, 0, crow, b, pol_c);
-                    ++n_c;
-                    if (++stage == S) { stage = 0; cph ^= 1u; }
+        // (all lanes wait, lane 0 issues; in resident mode the warp also computes the second
+        // half of each point tile's norms before handing the item's stages back)
+        const uint64_t pol_c = l2_policy_evict_last();
+        const uint32_t xaug_full_leader0 = map_to_rank(XAUG_FULL(0), 0);
+        const uint32_t xaug_full_leader1 = map_to_rank(XAUG_FULL(1), 0);
+        int stage = 0;
+        uint32_t cph = 0;
+        long long n_c = 0;
+        bool ok = true;
+        int cur_b = -1;   // batch element whose centroid tiles the ring holds (resident mode)
+        int local = 0;
+        for (int t = t_begin; t < t_end && ok; ++t, ++local) {
+            const int b = t / p.mtiles;
+            if (p.resident) {
+                const int xb = local & 1;
+                if (!mbar_wait_warp(X_FULL(xb), (local >> 1) & 1, abortp)) { ok = false; break; }
+                norm_rows(xb, local, BM / 2, BM);
+                if (lane == 0) {
+                    mbar_arrive_cluster(xb ? xaug_full_leader1 : xaug_full_leader0);
+                    mbar_arrive(DELTA_FULL(local & (DELTA_SLOTS - 1)));
+                    mbar_arrive(X_EMPTY(xb));
                 }
             }
-            if (!ok && leader) {
-                // Let every pair copy issued into the ring land before shared memory goes away
-                // (n_c counts every use of the ring, so each stage's last phase is known).
-                for (int s = 0; s < S; ++s) {
-                    const long long uses = n_c > s ? (n_c - 1 - s) / S + 1 : 0;
-                    if (uses) mbar_wait(C_FULL(s), static_cast<uint32_t>((uses - 1) & 1), nullptr);
+            // Resident mode (the ring holds every tile of a batch element: stage j = tile j):
+            // the tiles are loaded again only when the batch element changes; otherwise the
+            // stage's phase just advances.
+            const bool reload = !p.resident || b != cur_b;
+            cur_b = b;
+            for (int j = 0; j < p.nct; ++j) {
+                const int crow = j * BN + static_cast<int>(rank) * CROWS;
+                if (!mbar_wait_warp(C_EMPTY(stage), cph ^ 1u, abortp)) { ok = false; break; }
+                if (lane == 0) {
+                    if (!reload) {
+                        if (leader) mbar_arrive(C_FULL(stage));
+                    } else {
+                        if (leader) mbar_arrive_expect_tx(C_FULL(stage), stage_tx);
+                        const uint32_t sdst = sbase + L.c_off + stage * L.stage;
+                        const uint32_t lbar = map_to_rank(C_FULL(stage), 0);
+                        for (int kc = 0; kc < NKC; ++kc)
+                            tma_load_3d_pair(sdst + kc * CCHUNK, &tmC, lbar, kc * KC, crow, b, pol_c);
+                        tma_load_3d_pair(sdst + NKC * CCHUNK, &tmA, lbar, 0, crow, b, pol_c);
+                    }
                 }
+                __syncwarp();
+                ++n_c;
+                if (++stage == S) { stage = 0; cph ^= 1u; }
+            }
+        }
+        if (!ok && leader && lane == 0) {
+            // Let every pair copy issued into the ring land before shared memory goes away
+            // (n_c counts every use of the ring, so each stage's last phase is known).
+            for (int s = 0; s < S; ++s) {
+                const long long uses = n_c > s ? (n_c - 1 - s) / S + 1 : 0;
+                if (uses) mbar_wait(C_FULL(s), static_cast<uint32_t>((uses - 1) & 1), nullptr);
             }
         }
         __syncwarp();
@@ -452,7 +502,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const uint64_t pol_x = l2_policy_evict_first();
         // test-only fault switch (off by default): withhold the first point tile of pair 0
         const bool withhold = blockIdx.x == 0 && *reinterpret_cast<volatile int *>(&g_km_inject) == 1;
-        float *dbuf = reinterpret_cast<float *>(sgen + L.delta_off);
         const uint32_t xaug_full_leader0 = map_to_rank(XAUG_FULL(0), 0);
         const uint32_t xaug_full_leader1 = map_to_rank(XAUG_FULL(1), 0);
         int n_x = 0;
@@ -476,33 +525,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             // The tile's norms as soon as it lands (this warp has nothing else to do until the
             // next buffer is handed back at the end of the work item before this one).
             if (!mbar_wait_warp(X_FULL(xb), xph, abortp)) { ok = false; break; }
-#pragma unroll 2
-            for (int rr = 0; rr < BM / 32; ++rr) {
-                const int row = lane + rr * 32;
-                const float half_xn =
-                    0.5f * tile_row_sqnorm<T>(sgen + L.x_off + xb * NKC * XCHUNK, NKC, row);
-                // The split carries ||x||^2/2 raised by 2^-12 of itself. The accumulator is then
-                // d/2 + (about 2^-13 ||x||^2), positive even for a point on its centroid, since
-                // the two-piece split (2^-18 relative) and the fp32 reduction (below 2^-15
-                // ||x||^2) err by less. Keys of positive floats order ties by index the way the
-                // min expects (lowest index wins); delta takes the raise back out of the
-                // reported distance, and a constant per row cannot change the argmin.
-                const float tgt = fmaf(half_xn, 0x1p-12f, half_xn);
-                const float x1 = __bfloat162float(__float2bfloat16_rn(tgt));
-                const float x2 = __bfloat162float(__float2bfloat16_rn(tgt - x1));
-                dbuf[(local & (DELTA_SLOTS - 1)) * BM + row] = (half_xn - x1) - x2;
-                // Row of the point-side augmentation in the 32-byte-swizzled layout: the two
-                // 16-byte halves of rows 4..7 of every 8-row group trade places.
-                const uint4 data = make_uint4(pack_bf16x2(x1, x2), pack_bf16x2(1.f, 1.f),
-                                              pack_bf16x2(1.f, 0.f), 0u);
-                const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-                uint8_t *rp = sgen + L.xaug_off + xb * XAUG_BYTES + row * 32;
-                const int sw = (row >> 2) & 1;
-                *reinterpret_cast<uint4 *>(rp + 16 * sw) = data;
-                *reinterpret_cast<uint4 *>(rp + 16 * (1 - sw)) = zero;
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
+            norm_rows(xb, local, 0, BM / nnorm);
             if (lane == 0) {
                 mbar_arrive_cluster(xb ? xaug_full_leader1 : xaug_full_leader0);
                 mbar_arrive(DELTA_FULL(local & (DELTA_SLOTS - 1)));
