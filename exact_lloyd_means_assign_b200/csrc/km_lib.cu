@@ -746,10 +746,11 @@ km_status run_update_final(const void *X, km_dtype dt, const int32_t *ids, const
     const int64_t sntiles = ceil_div(N, stile);
     if (smem_bins) {
         // the scan folded into the scatter: slot reservations on a zeroed fill counter
-        const size_t smem = static_cast<size_t>(2 * K + 1 + stile) * 4;
+        const size_t smem = static_cast<size_t>(K <= SCATTER_SORT_K_MAX ? ((2 * K + 1 + 3) & ~3) + K + stile
+                                                                        : 2 * K + 1) * 4;
         if (cudaMemsetAsync(f.cursor, 0, static_cast<size_t>(B * K) * 4, st) != cudaSuccess ||
             cudaFuncSetAttribute(scatter_final_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (2 * SMEM_K_MAX + 1 + TILE) * 4) != cudaSuccess)
+                                 (2 * SMEM_K_MAX + 1) * 4) != cudaSuccess)
             return KM_ERR_CUDA;
         for (int64_t b0 = 0; b0 < B; b0 += kMaxGridY) {
             const int64_t nb = std::min<int64_t>(kMaxGridY, B - b0);

@@ -32,6 +32,9 @@ namespace upd {
 
 constexpr int TILE = 8192;          // points per histogram / scatter tile
 constexpr int TILE_THREADS = 512;
+constexpr int SCATTER_PPT = TILE / TILE_THREADS;   // points per thread of a scatter tile
+constexpr int SCATTER_SORT_K_MAX = 4096;           // tiles sorted in shared memory up to this K
+static_assert(TILE <= 8192 && SCATTER_SORT_K_MAX <= (1 << 18), "(cluster, point) packs in 31 bits");
 constexpr int SMEM_K_MAX = 16384;   // bins kept in shared memory
 constexpr int SCAN_THREADS = 1024;
 constexpr int SEG_THREADS = 256;
@@ -923,53 +926,22 @@ __global__ void __launch_bounds__(SCAN_THREADS)
     if (tid == 0) ob[K] = carry;
 }
 
-// The counting-sort scatter with the scan folded in (K <= SMEM_K_MAX; shared memory: 2K + 1 +
-// tile ints). Every block computes its problem's exclusive offsets of the counts in shared
-// memory, reserves each cluster of its tile a slot range at offs[k] + atomicAdd(fill[b, k],
-// h[k]) (fill zeroed beforehand) and ranks its points into it. The blocks of a problem also
-// share the per-cluster work scan_final_kernel does: tile 0 writes offsets[b, 0..K]; each block
-// zeroes the arrival counters of its share of the clusters and writes the outputs of the empty
-// ones there (C_new = C_prev, Cx, cn, a zero weight sum; in the moving-average form only
-// Nc <- (1 - alpha) Nc).
-template <typename T>
-__global__ void __launch_bounds__(TILE_THREADS)
-    scatter_final_kernel(const int32_t *__restrict__ ids, const int32_t *__restrict__ counts, int N,
-                         int K, int d, int tile, int32_t *__restrict__ fill,
-                         int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
-                         int32_t *__restrict__ arrive, const float *C_prev, float *C_new,
-                         T *__restrict__ Cx, float *__restrict__ cn, float *__restrict__ wsum,
-                         float *__restrict__ Nc, float alpha, int range, int rpb,
-                         int32_t *__restrict__ rseg) {
+// Exclusive scan in place of a[0..K) (shared, 16-byte aligned) by one block of TILE_THREADS
+// threads; returns the total. 4 * TILE_THREADS entries per pass: thread t takes 4 consecutive
+// entries with one 16-byte access (a warp reads 512 contiguous bytes: no bank conflicts).
+__device__ __forceinline__ int block_exscan(int *a, int K, int *wtot) {
     constexpr int NW = TILE_THREADS / 32;
-    extern __shared__ __align__(16) int ssm[];
-    int *offs = ssm;             // [K + 1]: the counts, then their exclusive prefix
-    int *h = ssm + K + 1;        // [K]: the tile's histogram, then its reserved slot cursors
-    int *tids = h + K;           // [tile]: the tile's labels
-    __shared__ int wtot[NW];
-    const int b = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int t0 = blockIdx.x * tile;
-    const int t1 = min(N, t0 + tile);
-    const int64_t kb = static_cast<int64_t>(b) * K;
-    const int32_t *idb = ids + static_cast<int64_t>(b) * N;
-    for (int k = tid; k < K; k += TILE_THREADS) {
-        offs[k] = counts[kb + k];
-        h[k] = 0;
-    }
-    for (int i = t0 + tid; i < t1; i += TILE_THREADS) tids[i - t0] = idb[i];
-    __syncthreads();
-    // exclusive scan in place, 4 * TILE_THREADS counts per pass: thread t takes 4 consecutive
-    // counts with one 16-byte access (a warp reads 512 contiguous bytes: no bank conflicts)
     int carry = 0;
     for (int base = 0; base < K; base += 4 * TILE_THREADS) {
         const int kk = base + 4 * tid;
         int v[4];
         if (kk + 3 < K) {
-            const int4 q = *reinterpret_cast<const int4 *>(offs + kk);
+            const int4 q = *reinterpret_cast<const int4 *>(a + kk);
             v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
         } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) v[e] = kk + e < K ? offs[kk + e] : 0;
+            for (int e = 0; e < 4; ++e) v[e] = kk + e < K ? a[kk + e] : 0;
         }
         const int tsum = v[0] + v[1] + v[2] + v[3];
         int incl = tsum;
@@ -998,21 +970,72 @@ __global__ void __launch_bounds__(TILE_THREADS)
             ex += v[e];
         }
         if (kk + 3 < K) {
-            *reinterpret_cast<int4 *>(offs + kk) = make_int4(o4[0], o4[1], o4[2], o4[3]);
+            *reinterpret_cast<int4 *>(a + kk) = make_int4(o4[0], o4[1], o4[2], o4[3]);
         } else {
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-                if (kk + e < K) offs[kk + e] = o4[e];
+                if (kk + e < K) a[kk + e] = o4[e];
         }
         carry += wtot[NW - 1];
         __syncthreads();
     }
-    if (tid == 0) offs[K] = carry;
-    // the tile's histogram
-    for (int i = tid; i < t1 - t0; i += TILE_THREADS) {
-        const int k = tids[i];
-        if (static_cast<unsigned>(k) < static_cast<unsigned>(K)) atomicAdd(&h[k], 1);
+    return carry;
+}
+
+// The counting-sort scatter with the scan folded in (K <= SMEM_K_MAX; tile <= SCATTER_PPT *
+// TILE_THREADS, each thread keeping its points' labels in registers so the tile's histogram and
+// ranking issue all their shared-memory atomics back to back). With K <= SCATTER_SORT_K_MAX the
+// tile is first sorted by cluster in shared memory (a tile-local scan of its histogram, then
+// cursors), and perm is written in that order: each cluster's run of the tile leaves as
+// contiguous stores instead of one scattered 4-byte store per point. Shared memory: 2K + 1 ints,
+// plus (sorted form) K + tile ints from a 16-byte boundary. Every block computes its problem's exclusive offsets of the counts in shared
+// memory, reserves each cluster of its tile a slot range at offs[k] + atomicAdd(fill[b, k],
+// h[k]) (fill zeroed beforehand) and ranks its points into it. The blocks of a problem also
+// share the per-cluster work scan_final_kernel does: tile 0 writes offsets[b, 0..K]; each block
+// zeroes the arrival counters of its share of the clusters and writes the outputs of the empty
+// ones there (C_new = C_prev, Cx, cn, a zero weight sum; in the moving-average form only
+// Nc <- (1 - alpha) Nc).
+template <typename T>
+__global__ void __launch_bounds__(TILE_THREADS)
+    scatter_final_kernel(const int32_t *__restrict__ ids, const int32_t *__restrict__ counts, int N,
+                         int K, int d, int tile, int32_t *__restrict__ fill,
+                         int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
+                         int32_t *__restrict__ arrive, const float *C_prev, float *C_new,
+                         T *__restrict__ Cx, float *__restrict__ cn, float *__restrict__ wsum,
+                         float *__restrict__ Nc, float alpha, int range, int rpb,
+                         int32_t *__restrict__ rseg) {
+    constexpr int NW = TILE_THREADS / 32;
+    extern __shared__ __align__(16) int ssm[];
+    int *offs = ssm;             // [K + 1]: the counts, then their exclusive prefix
+    int *h = ssm + K + 1;        // [K]: the tile's histogram, then its reserved slots
+    const bool sorted_form = K <= SCATTER_SORT_K_MAX;
+    int *lofs = ssm + ((2 * K + 1 + 3) & ~3);   // [K] (sorted form): the histogram's prefix, then cursors
+    int *srt = lofs + K;                        // [tile] (sorted form): (cluster, point) by cluster
+    __shared__ int wtot[NW];
+    const int b = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int t0 = blockIdx.x * tile;
+    const int t1 = min(N, t0 + tile);
+    const int64_t kb = static_cast<int64_t>(b) * K;
+    const int32_t *idb = ids + static_cast<int64_t>(b) * N;
+    // this thread's points t0 + tid + m * TILE_THREADS: labels loaded first, all in flight
+    int lab[SCATTER_PPT];
+#pragma unroll
+    for (int m = 0; m < SCATTER_PPT; ++m) {
+        const int i = t0 + tid + m * TILE_THREADS;
+        lab[m] = i < t1 ? idb[i] : -1;
     }
+    for (int k = tid; k < K; k += TILE_THREADS) {
+        offs[k] = counts[kb + k];
+        h[k] = 0;
+    }
+    __syncthreads();
+    const int total = block_exscan(offs, K, wtot);
+    if (tid == 0) offs[K] = total;
+    // the tile's histogram
+#pragma unroll
+    for (int m = 0; m < SCATTER_PPT; ++m)
+        if (static_cast<unsigned>(lab[m]) < static_cast<unsigned>(K)) atomicAdd(&h[lab[m]], 1);
     __syncthreads();
     // this problem's per-cluster work, split over its tiles
     if (blockIdx.x == 0) {
@@ -1056,15 +1079,37 @@ __global__ void __launch_bounds__(TILE_THREADS)
             if (wsum && lane == 0) wsum[row] = 0.f;
         }
     }
+    int32_t *pb = perm + static_cast<int64_t>(b) * N;
+    if (sorted_form) {
+        for (int k = tid; k < K; k += TILE_THREADS) lofs[k] = h[k];
+        __syncthreads();
+        const int nvalid = block_exscan(lofs, K, wtot);
+        // each cluster's slot range, kept as (global slot - tile-local position)
+        for (int k = tid; k < K; k += TILE_THREADS)
+            if (h[k]) h[k] = offs[k] + atomicAdd(&fill[kb + k], h[k]) - lofs[k];
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < SCATTER_PPT; ++m)
+            if (static_cast<unsigned>(lab[m]) < static_cast<unsigned>(K))
+                srt[atomicAdd(&lofs[lab[m]], 1)] = (lab[m] << 13) | (tid + m * TILE_THREADS);
+        __syncthreads();
+        for (int lp = tid; lp < nvalid; lp += TILE_THREADS) {
+            const int e = srt[lp];
+            pb[lp + h[e >> 13]] = t0 + (e & 8191);
+        }
+        return;
+    }
     // reserve each cluster of the tile a slot range, then rank the points into it
     for (int k = tid; k < K; k += TILE_THREADS)
         if (h[k]) h[k] = offs[k] + atomicAdd(&fill[kb + k], h[k]);
     __syncthreads();
-    int32_t *pb = perm + static_cast<int64_t>(b) * N;
-    for (int i = tid; i < t1 - t0; i += TILE_THREADS) {
-        const int k = tids[i];
-        if (static_cast<unsigned>(k) < static_cast<unsigned>(K)) pb[atomicAdd(&h[k], 1)] = t0 + i;
-    }
+    int pos[SCATTER_PPT];
+#pragma unroll
+    for (int m = 0; m < SCATTER_PPT; ++m)
+        pos[m] = static_cast<unsigned>(lab[m]) < static_cast<unsigned>(K) ? atomicAdd(&h[lab[m]], 1) : -1;
+#pragma unroll
+    for (int m = 0; m < SCATTER_PPT; ++m)
+        if (pos[m] >= 0) pb[pos[m]] = t0 + tid + m * TILE_THREADS;
 }
 
 }  // namespace upd
