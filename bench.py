@@ -101,6 +101,14 @@ def _profile_traffic(name="assign_tc_batched_assign_bound.md", files=("km_assign
     return float(m.group(1))
 
 
+def lloyd_roofline(flop, update_bytes, ms_per_iter, peak_tf, peak_gbs):
+    """Whole-iteration roofline: the time the assignment's contraction takes at the tensor peak
+    plus the time the update's algorithmic bytes take at the HBM peak, over the measured time."""
+    ideal_ms = flop / (peak_tf * 1e12) * 1e3 + update_bytes / (peak_gbs * 1e9) * 1e3
+    return {"ideal_ms": ideal_ms, "measured_ms": ms_per_iter, "frac": ideal_ms / ms_per_iter,
+            "definition": "(flop / tensor peak + update bytes / HBM peak) / time per iteration"}
+
+
 class ClockSampler:
     """nvidia-smi clock/throttle sampling while the timed region runs."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -419,6 +427,7 @@ def run_gpu(args):
             "update_roofline": {"bound": "hbm", "achieved": upd_gbs, "peak": peak_bw, "unit": "GB/s",
                                 "frac": upd_gbs / peak_bw, "algorithmic_bytes": UPDATE_BYTES,
                                 "peak_source": peak_kind},
+            "lloyd_roofline": lloyd_roofline(ASSIGN_FLOP, UPDATE_BYTES, ms_step, peak_tf, peak_bw),
             "e2e": {"value": ws * 1e3 / e2e_ms, "unit": "iter/s",
                     "h2d_bytes_per_step": B * N * D * 2 + B * K * D * 4,
                     "d2h_bytes_per_step": B * K * D * 4 + B * 8},
@@ -683,6 +692,7 @@ def run_workload(args):
                                      "peak": peak_bw, "unit": "GB/s",
                                      "frac": ubytes / (u_ms * 1e-3) / 1e9 / peak_bw,
                                      "algorithmic_bytes": ubytes, "peak_source": peak_kind},
+                    lloyd_roofline=lloyd_roofline(flop, ubytes, ms, peak_tf, peak_bw),
                     gpu_launches=LAUNCHES_PER_STEP * args.steps * blocks, clocks=clk.summary(),
                     device_error=km.km_device_error())
         if cpu:
