@@ -103,4 +103,31 @@ __global__ void caug_kernel(const T *__restrict__ Cx, const float *__restrict__ 
     }
 }
 
+// The same rows from given norms, one thread per row (two 16-byte stores): the warp-per-row form
+// above is only needed when the norms must be summed from Cx.
+__global__ void caug_rows_kernel(const float *__restrict__ cn, int B, int K, int Kp,
+                                 __nv_bfloat16 *__restrict__ caug) {
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (row >= static_cast<int64_t>(B) * Kp) return;
+    const int b = static_cast<int>(row / Kp), k = static_cast<int>(row % Kp);
+    __nv_bfloat16 e[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) e[j] = __float2bfloat16_rn(0.f);
+    if (k >= K) {
+        e[2] = __float2bfloat16_rn(1e30f);   // a padding column can never win
+    } else {
+        const float h = 0.5f * cn[static_cast<int64_t>(b) * K + k];
+        const float a = __bfloat162float(__float2bfloat16_rn(h));
+        const float r1 = h - a;
+        const float b2 = __bfloat162float(__float2bfloat16_rn(r1));
+        e[0] = e[1] = __float2bfloat16_rn(1.f);
+        e[2] = __float2bfloat16_rn(a);
+        e[3] = __float2bfloat16_rn(b2);
+        e[4] = __float2bfloat16_rn(r1 - b2);
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(caug + row * 16);
+    dst[0] = *reinterpret_cast<const uint4 *>(&e[0]);
+    dst[1] = *reinterpret_cast<const uint4 *>(&e[8]);
+}
+
 }  // namespace km

@@ -373,9 +373,14 @@ km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float 
     const int bn = tc_bn(K, d);
     const int64_t Kp = tc_kp(K, d);
     const int nkc = static_cast<int>(ceil_div(d, KC));
-    km::caug_kernel<T><<<static_cast<unsigned>(ceil_div(B * Kp, 8)), 256, 0, st>>>(
-        static_cast<const T *>(Cx), cn, static_cast<int>(B), static_cast<int>(K),
-        static_cast<int>(Kp), static_cast<int>(d), static_cast<__nv_bfloat16 *>(caug));
+    if (cn && aligned(caug, 16))
+        km::caug_rows_kernel<<<static_cast<unsigned>(ceil_div(B * Kp, 256)), 256, 0, st>>>(
+            cn, static_cast<int>(B), static_cast<int>(K), static_cast<int>(Kp),
+            static_cast<__nv_bfloat16 *>(caug));
+    else
+        km::caug_kernel<T><<<static_cast<unsigned>(ceil_div(B * Kp, 8)), 256, 0, st>>>(
+            static_cast<const T *>(Cx), cn, static_cast<int>(B), static_cast<int>(K),
+            static_cast<int>(Kp), static_cast<int>(d), static_cast<__nv_bfloat16 *>(caug));
     if (launch_status() != KM_OK) return KM_ERR_CUDA;
 
     const CUtensorMapDataType tdt =
