@@ -577,7 +577,10 @@ def run_workload(args):
                           eager_us_per_iter=eager * 1e3 / iters,
                           config={"workload": wl.name, "B": Bw, "N": Nw, "K": Kw, "d": Dw,
                                   "iterations_per_step": iters, "launch": "CUDA graph of one km_fit call"},
-                          roofline={"bound": "latency", "note": "4.2 MFLOP per iteration; launch-bound"},
+                          roofline={"bound": "latency",
+                                    "note": "4.2 MFLOP per iteration; the whole fit is one cooperative "
+                                            "launch (fit_small_kernel) with one grid barrier per iteration"},
+                          gpu_launches=args.steps * blocks,
                           cpu_baseline={"value": cpu_s * 1e6 / iters, "unit": "us/iter",
                                         "cores": oracle.threads(), "kind": "oracle",
                                         "sample": f"the whole fit ({iters} iterations, fp64), {cpu_s:.2f} s"},

@@ -21,6 +21,7 @@
 #include "km_common.cuh"
 #include "km_emeans.cuh"
 #include "km_fit1d.cuh"
+#include "km_fit_small.cuh"
 #include "km_update.cuh"
 
 namespace {
@@ -142,6 +143,33 @@ inline Fit1dWs carve_fit1d(Carver &c, int64_t B, int64_t N) {
     return g;
 }
 
+// Whole-fit single launch for small problems (km_fit_small.cuh): shapes it may take. The launch
+// itself is used only when every CTA can be resident at once (checked at run time).
+constexpr int64_t kSmallMaxCtas = 2048;
+inline bool fit_small_shape_ok(int64_t B, int64_t N, int64_t K, int64_t d) {
+    return d >= 1 && d <= 64 && K * d <= 4096 && B * ceil_div(N, km::fs::kPts) <= kSmallMaxCtas &&
+           B * N * K * d <= (int64_t{1} << 27);
+}
+// One block, zeroed before each launch: three accumulators [3, B, K, d + 2] fp32, three inertia
+// slots [3, B] fp64, the barrier words.
+struct SmallWs {
+    float *acc;
+    double *iacc;
+    unsigned int *bar;
+    size_t bytes;
+};
+inline SmallWs carve_small(Carver &c, int64_t B, int64_t K, int64_t d) {
+    const size_t abytes = static_cast<size_t>(3 * B * K * (d + 2)) * 4;
+    const size_t ibytes = static_cast<size_t>(3 * B) * 8;
+    SmallWs s;
+    s.bytes = align_up(abytes) + align_up(ibytes) + 16;
+    uint8_t *base = c.take<uint8_t>(s.bytes);
+    s.acc = reinterpret_cast<float *>(base);
+    s.iacc = base ? reinterpret_cast<double *>(base + align_up(abytes)) : nullptr;
+    s.bar = base ? reinterpret_cast<unsigned int *>(base + align_up(abytes) + align_up(ibytes)) : nullptr;
+    return s;
+}
+
 struct FitWs {
     void *Cx;
     float *cn;
@@ -159,7 +187,9 @@ inline FitWs carve_fit(Carver &c, int64_t B, int64_t N, int64_t K, int64_t d, km
     f.rest = c.base ? c.base + c.off : nullptr;
     Carver g(nullptr);
     if (fit1d_rows_ok(N, K, d)) carve_fit1d(g, B, N);
-    c.off += std::max({ws_update(B, N, K, d), ws_assign(B, K, d, dt), g.off});
+    Carver h(nullptr);
+    if (fit_small_shape_ok(B, N, K, d)) carve_small(h, B, K, d);
+    c.off += std::max({ws_update(B, N, K, d), ws_assign(B, K, d, dt), g.off, h.off});
     return f;
 }
 
@@ -902,6 +932,64 @@ km_status run_fit1d(const void *X, const float *w, int64_t B, int64_t N, int64_t
     return launch_status();
 }
 
+// The whole fit in one cooperative launch (km_fit_small.cuh). Returns KM_ERR_UNSUPPORTED, with
+// nothing enqueued, when the CTAs could not all be resident at once.
+template <typename T, int DM>
+km_status run_fit_small(const void *X, const float *w, int64_t B, int64_t N, int64_t K, int64_t d,
+                        float *C, int iters, int32_t *ids, double *inertia_hist, float *C_hist,
+                        void *rest, cudaStream_t st) {
+    Carver c(rest);
+    SmallWs sw = carve_small(c, B, K, d);
+    km::fs::Params p;
+    p.B = static_cast<int>(B);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.d = static_cast<int>(d);
+    p.P = static_cast<int>(ceil_div(N, km::fs::kPts));
+    p.iters = iters;
+    p.w = w;
+    p.C = C;
+    p.ids = ids;
+    p.inertia_hist = inertia_hist;
+    p.C_hist = C_hist;
+    p.acc = sw.acc;
+    p.iacc = sw.iacc;
+    p.bar = sw.bar;
+    const size_t smem = static_cast<size_t>(2 * K * d + km::fs::kPts * (d + 3) + K + 1) * 4;
+    if (cudaFuncSetAttribute(km::fs::fit_small_kernel<T, DM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return KM_ERR_CUDA;
+    const int ctas = static_cast<int>(B) * p.P;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, km::fs::fit_small_kernel<T, DM>,
+                                                      km::fs::kThreads, smem) != cudaSuccess)
+        return KM_ERR_CUDA;
+    if (static_cast<int64_t>(per_sm) * num_sms() < ctas) return KM_ERR_UNSUPPORTED;
+    if (cudaMemsetAsync(sw.acc, 0, sw.bytes, st) != cudaSuccess) return KM_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+    cfg.blockDim = dim3(km::fs::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;   // every CTA resident: the grid barrier needs it
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, km::fs::fit_small_kernel<T, DM>, static_cast<const T *>(X), p) != cudaSuccess)
+        return KM_ERR_CUDA;
+    return launch_status();
+}
+
+template <typename T>
+km_status fit_small_dispatch(const void *X, const float *w, int64_t B, int64_t N, int64_t K, int64_t d,
+                             float *C, int iters, int32_t *ids, double *inertia_hist, float *C_hist,
+                             void *rest, cudaStream_t st) {
+    if (d <= 16) return run_fit_small<T, 16>(X, w, B, N, K, d, C, iters, ids, inertia_hist, C_hist, rest, st);
+    if (d <= 32) return run_fit_small<T, 32>(X, w, B, N, K, d, C, iters, ids, inertia_hist, C_hist, rest, st);
+    return run_fit_small<T, 64>(X, w, B, N, K, d, C, iters, ids, inertia_hist, C_hist, rest, st);
+}
+
 km_status do_fit(const void *X, km_dtype dt, const float *w, int64_t B, int64_t N, int64_t K,
                  int64_t d, float *C, int iters, int32_t *ids, double *inertia_hist, float *C_hist,
                  void *ws, cudaStream_t st) {
@@ -914,6 +1002,15 @@ km_status do_fit(const void *X, km_dtype dt, const float *w, int64_t B, int64_t 
             default:
                 return run_fit1d<__nv_bfloat16>(X, w, B, N, K, C, iters, ids, inertia_hist, C_hist, f.rest, st);
         }
+    }
+    if (fit_small_shape_ok(B, N, K, d) && iters > 0 && aligned(X, dtype_size(dt))) {
+        km_status s = KM_ERR_UNSUPPORTED;
+        switch (dt) {
+            case KM_F32: s = fit_small_dispatch<float>(X, w, B, N, K, d, C, iters, ids, inertia_hist, C_hist, f.rest, st); break;
+            case KM_F16: s = fit_small_dispatch<__half>(X, w, B, N, K, d, C, iters, ids, inertia_hist, C_hist, f.rest, st); break;
+            default: s = fit_small_dispatch<__nv_bfloat16>(X, w, B, N, K, d, C, iters, ids, inertia_hist, C_hist, f.rest, st);
+        }
+        if (s != KM_ERR_UNSUPPORTED) return s;   // else: the step-by-step fit below
     }
     void *caug = f.rest;  // assignment scratch shares the update region (used one after the other)
     const bool fused = final_ok(dt, X, B, N, d);
@@ -1578,7 +1675,7 @@ km_status km_debug_wait_limit(unsigned long long limit_ns, unsigned long long *p
 }
 
 km_status km_debug_inject(int mode) {
-    if (mode != 0 && mode != 1) return KM_ERR_INVALID_ARG;
+    if (mode < 0 || mode > 2) return KM_ERR_INVALID_ARG;
     if (cudaDeviceSynchronize() != cudaSuccess ||
         cudaMemcpyToSymbol(km::g_km_inject, &mode, sizeof(mode)) != cudaSuccess)
         return KM_ERR_CUDA;

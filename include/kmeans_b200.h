@@ -198,7 +198,12 @@ km_status km_init_grid1d(const void *X, km_dtype dtype, int64_t B, int64_t N, in
  * kernel sorts every row once and stores the sorted values, indices and fp64 prefix sums of w,
  * w*x, w*x^2 in the workspace (32 bytes per point), then one kernel runs all iterations with a
  * warp per row; for 32 < K <= 64 one fused kernel per row keeps the row on chip (no workspace
- * needed). Everything else chains km_prep / km_assign / km_update on the stream. `ws` must hold
+ * needed). Small problems (K * d <= 4096, d <= 64, B * ceil(N / 256) <= 2048 CTAs that can all
+ * be resident, B * N * K * d <= 2^27, iters > 0) run the whole fit in one cooperative launch:
+ * each CTA keeps 256 points in registers and assigns them with the same fp32 direct-form
+ * arithmetic as the CUDA-core assignment, per-CTA partial sums are combined in CTA order after
+ * a grid barrier whose waits are bounded like every other wait of the library. Everything else
+ * chains km_prep / km_assign / km_update on the stream. `ws` must hold
  * km_workspace_size(KM_OP_FIT, ...) bytes (else KM_ERR_WORKSPACE).
  */
 km_status km_fit(const void *X, km_dtype dtype, const float *w, int64_t B, int64_t N, int64_t K,
@@ -255,8 +260,11 @@ km_status km_device_error(void *stream, int *code);
  * first SM pair: the waits on it run out, every role of that pair leaves its loop, copies in
  * flight land, the issued MMAs drain, tensor memory is freed and the kernel returns with bit 0
  * of the device error word set (km_device_error reports KM_ERR_DEVICE_TIMEOUT); its labels
- * are left unwritten. km_debug_inject(0) (the default) turns it off. Both synchronise the device
- * first. No fault, trap or endless loop is involved.
+ * are left unwritten. km_debug_inject(2) makes the first CTA of the next single-launch small fits
+ * (km_fit on shapes with K * d <= 4096, d <= 64 and at most 2048 CTAs of 256 points) skip its
+ * first grid-barrier arrival: the other CTAs' waits run out, set bit 0 and an abort word, and
+ * every CTA leaves. km_debug_inject(0) (the default) turns both off. Both calls synchronise the
+ * device first. No fault, trap or endless loop is involved.
  */
 km_status km_debug_wait_limit(unsigned long long limit_ns, unsigned long long *previous_ns);
 km_status km_debug_inject(int mode);
