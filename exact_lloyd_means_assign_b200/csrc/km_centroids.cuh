@@ -105,11 +105,16 @@ __global__ void caug_kernel(const T *__restrict__ Cx, const float *__restrict__ 
 
 // The same rows from given norms, one thread per row (two 16-byte stores): the warp-per-row form
 // above is only needed when the norms must be summed from Cx.
+// It also clears the assignment's per-cluster counts and per-problem objective when given (the
+// assignment that follows adds into them), saving two memset launches per assignment.
 __global__ void caug_rows_kernel(const float *__restrict__ cn, int B, int K, int Kp,
-                                 __nv_bfloat16 *__restrict__ caug) {
+                                 __nv_bfloat16 *__restrict__ caug, int32_t *__restrict__ zero_counts,
+                                 double *__restrict__ zero_inertia) {
     const int64_t row = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (row >= static_cast<int64_t>(B) * Kp) return;
     const int b = static_cast<int>(row / Kp), k = static_cast<int>(row % Kp);
+    if (zero_counts && k < K) zero_counts[static_cast<int64_t>(b) * K + k] = 0;
+    if (zero_inertia && row < B) zero_inertia[row] = 0.0;
     __nv_bfloat16 e[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) e[j] = __float2bfloat16_rn(0.f);

@@ -396,7 +396,8 @@ template <typename T>
 km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float *cn,
                         const float *w, int64_t B, int64_t N, int64_t K, int64_t d, int32_t *ids,
                         float *mind, double *inertia, int32_t *counts, void *caug, int64_t xld,
-                        cudaStream_t st) {
+                        cudaStream_t st, int32_t *zero_counts = nullptr,
+                        double *zero_inertia = nullptr) {
     using namespace km::tc;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return KM_ERR_CUDA;
@@ -406,7 +407,7 @@ km_status run_assign_tc(const void *X, km_dtype dt, const void *Cx, const float 
     if (cn && aligned(caug, 16))
         km::caug_rows_kernel<<<static_cast<unsigned>(ceil_div(B * Kp, 256)), 256, 0, st>>>(
             cn, static_cast<int>(B), static_cast<int>(K), static_cast<int>(Kp),
-            static_cast<__nv_bfloat16 *>(caug));
+            static_cast<__nv_bfloat16 *>(caug), zero_counts, zero_inertia);
     else
         km::caug_kernel<T><<<static_cast<unsigned>(ceil_div(B * Kp, 8)), 256, 0, st>>>(
             static_cast<const T *>(Cx), cn, static_cast<int>(B), static_cast<int>(K),
@@ -494,19 +495,25 @@ km_status do_assign(const void *X, km_dtype dt, const void *Cx, const float *cn,
                     double *inertia, void *caug, cudaStream_t st, bool accumulate_inertia = false,
                     int32_t *counts = nullptr, int64_t xld = 0) {
     if (xld == 0) xld = N;
-    if (inertia && !accumulate_inertia &&
-        cudaMemsetAsync(inertia, 0, static_cast<size_t>(B) * 8, st) != cudaSuccess)
-        return KM_ERR_CUDA;
-    if (counts && cudaMemsetAsync(counts, 0, static_cast<size_t>(B * K) * 4, st) != cudaSuccess)
-        return KM_ERR_CUDA;
     const bool tc = tc_shape_ok(dt, d) && aligned(X, 16) && aligned(Cx, 16) && caug != nullptr &&
                     B * ceil_div(N, 128) <= kMaxIndex;
+    double *zero_inertia = inertia && !accumulate_inertia ? inertia : nullptr;
+    // the tensor-core path's augmentation kernel clears the counts and the objective itself
+    const bool folded = tc && cn && aligned(caug, 16);
+    if (!folded) {
+        if (zero_inertia && cudaMemsetAsync(zero_inertia, 0, static_cast<size_t>(B) * 8, st) != cudaSuccess)
+            return KM_ERR_CUDA;
+        if (counts && cudaMemsetAsync(counts, 0, static_cast<size_t>(B * K) * 4, st) != cudaSuccess)
+            return KM_ERR_CUDA;
+    }
     if (tc) {
+        int32_t *zc = folded ? counts : nullptr;
+        double *zi = folded ? zero_inertia : nullptr;
         if (dt == KM_F16)
             return run_assign_tc<__half>(X, dt, Cx, cn, w, B, N, K, d, ids, mind, inertia, counts, caug,
-                                         xld, st);
+                                         xld, st, zc, zi);
         return run_assign_tc<__nv_bfloat16>(X, dt, Cx, cn, w, B, N, K, d, ids, mind, inertia, counts,
-                                            caug, xld, st);
+                                            caug, xld, st, zc, zi);
     }
     switch (dt) {
         case KM_F32: return run_assign_simt<float>(X, Cx, w, B, N, K, d, ids, mind, inertia, counts, xld, st);
