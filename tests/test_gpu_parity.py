@@ -234,6 +234,8 @@ UPD_CASES = [
     ("f32", 1, 1000, 10, 32),
     ("bf16", 40, 700, 30, 64),       # more problems than ranges per problem
     ("f16", 1, 30000, 20000, 128),   # K above the 16384 shared-memory bins: the two-launch sort
+    ("f16", 2, 20000, 4096, 128),    # the largest K whose scatter tiles are sorted in shared memory
+    ("bf16", 1, 20000, 4097, 64),    # one above: labels ranked straight into perm
 ]
 
 
