@@ -260,7 +260,19 @@ def timed_blocks(phases, steps, stream, pg=None, min_s=MIN_TIMED_S):
         t_total += blk * 1e-3
         if len(per_block) == 1:
             need = max(3, math.ceil(min_s / max(blk * 1e-3, 1e-6)))
+            # every rank must run the same number of blocks (each starts with a barrier)
+            need = _agree_max(need, pg)
     return _median(per_block), [_median(p) for p in per_phase], len(per_block)
+
+
+def _agree_max(n, pg):
+    """The largest of the ranks' values of n (n itself with one process)."""
+    if not pg:
+        return n
+    dev = "cpu" if pg.get_backend() == "gloo" else torch.device("cuda", torch.cuda.current_device())
+    t = torch.tensor([n], dtype=torch.int64, device=dev)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return int(t.item())
 
 
 def _max_over_ranks(vals, pg, dev):

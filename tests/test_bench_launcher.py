@@ -53,3 +53,30 @@ def test_median_and_update_bytes():
     assert bench._median([4.0, 1.0, 2.0, 3.0]) == 2.5
     # the survey's algorithmic bytes of the headline update: X once + 4 passes over int32 ids
     assert bench.UPDATE_BYTES == 32 * 65536 * 128 * 2 + 4 * 32 * 65536 * 4
+
+
+def _agree_rank(rank, port, out):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=2)
+    try:
+        # the ranks' own block counts differ; every rank must run the larger one
+        out[rank] = bench._agree_max(3 + 2 * rank, dist)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ranks_agree_on_the_number_of_timed_blocks():
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        port = bench._free_port()
+        ps = [ctx.Process(target=_agree_rank, args=(r, port, out)) for r in range(2)]
+        for p in ps:
+            p.start()
+        for p in ps:
+            p.join(120)
+        assert all(p.exitcode == 0 for p in ps)
+        assert dict(out) == {0: 5, 1: 5}
+    assert bench._agree_max(7, None) == 7
