@@ -286,8 +286,9 @@ template <> struct SortKey<__nv_bfloat16> : SortKey16<__nv_bfloat16, 0> {
 // Stable LSD radix sort of one row in shared memory, 8-bit digits (2 passes for 16-bit values, 4
 // for fp32), by the block's THREADS threads. Warp w owns the contiguous positions
 // [w * seg, (w + 1) * seg) and walks them 32 at a time: lanes holding the same digit find each
-// other with a match, take consecutive slots after the warp's running count for that digit, and
-// the lowest of them advances the count. A block-wide scan over (digit, warp) then turns the
+// other (eight ballots, one per digit bit), take consecutive slots after the warp's running
+// count for that digit, and the lowest of them advances the count. A block-wide scan over
+// (digit, warp) then turns the
 // per-warp counts into destinations. Equal keys keep their order, so ties stay in index order.
 // Padding positions carry the largest key and sort to the end. Result in (ka, ia).
 constexpr int RADIX_WARPS = THREADS / 32;
@@ -308,7 +309,14 @@ __device__ __forceinline__ void radix_sort_row(Word *ka, uint16_t *ia, Word *kb,
             if (r < rounds) {
                 const int pos = warp * seg + r * 32 + lane;
                 const int dg = (ka[pos] >> shift) & 255;
-                const unsigned m = __match_any_sync(0xffffffffu, dg);
+                // the lanes holding the same digit: those agreeing on all eight bits (eight
+                // ballots; measured faster here than one match instruction)
+                unsigned m = 0xffffffffu;
+#pragma unroll
+                for (int bit = 0; bit < 8; ++bit) {
+                    const unsigned bal = __ballot_sync(0xffffffffu, (dg >> bit) & 1);
+                    m &= ((dg >> bit) & 1) ? bal : ~bal;
+                }
                 const int base = hist[warp][dg];
                 local[r] = base + __popc(m & lt);
                 __syncwarp();
