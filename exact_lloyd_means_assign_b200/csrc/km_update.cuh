@@ -586,27 +586,48 @@ __device__ __forceinline__ void finalize_one(const FinalParams &p, int64_t row, 
 // at the start, after every step and after a split):
 //     Nc' = (1 - a) Nc + a n,   C' = ((1 - a) Nc C + a s) / Nc'   (C kept when Nc' == 0);
 // Cx and cn follow C', and the batch statistics are added to the epoch totals.
+//
+// The cluster's state before this batch (count, centroid slice, epoch sum slice) is loaded when
+// the warp meets the cluster's first row, so the loads run under its accumulation; only the
+// finalizing warp uses them and nothing writes them before that finalize.
+template <int V>
+struct EmaPre {
+    float nold;
+    float c[V], es[V];
+};
+template <typename T, int V>
+__device__ __forceinline__ void ema_prefetch(const FinalParams &p, int64_t row, int lane, EmaPre<V> &q) {
+    constexpr int D = 32 * V;
+    const int64_t e0 = row * D + lane * V;
+    q.nold = p.Nc[row];
+#pragma unroll
+    for (int e = 0; e < V; ++e) {
+        q.c[e] = p.C_new[e0 + e];
+        q.es[e] = p.eS ? p.eS[e0 + e] : 0.f;
+    }
+}
+
 template <typename T, int V>
 __device__ __forceinline__ void finalize_ema(const FinalParams &p, int64_t row, int lane,
                                              const float (&s)[V], float wacc, int cnt,
-                                             bool weighted) {
+                                             bool weighted, const EmaPre<V> &q) {
     constexpr int D = 32 * V;
     const float a = p.alpha, a1 = 1.f - a;
     const float n = weighted ? wacc : static_cast<float>(cnt);
-    const float nold = p.Nc[row];
+    const float nold = q.nold;
     const float nn = a1 * nold + a * n;
     const int64_t e0 = row * D + lane * V;
     float sq = 0.f;
 #pragma unroll
     for (int e = 0; e < V; ++e) {
-        const float c = p.C_new[e0 + e];
+        const float c = q.c[e];
         const float v = nn > 0.f ? (a1 * nold * c + a * s[e]) / nn : c;
         p.C_new[e0 + e] = v;
         const T t = Cvt<T>::from_f(v);
         static_cast<T *>(p.Cx)[e0 + e] = t;
         const float f = Cvt<T>::to_f(t);
         sq = fmaf(f, f, sq);
-        if (p.eS) p.eS[e0 + e] += s[e];
+        if (p.eS) p.eS[e0 + e] = q.es[e] + s[e];
     }
     sq = warp_sum(sq);
     if (lane == 0) {
@@ -696,11 +717,12 @@ __global__ void __launch_bounds__(fz_warps(32 * V * sizeof(T)) * 32, 1)
     for (int e = 0; e < V; ++e) acc[e] = 0.f;
     float wacc = 0.f;
     int acck = -1, seg_s = 0, seg_e = 0;
+    EmaPre<V> pre;   // the moving-average form's prefetched cluster state
 
     auto flush = [&]() {
         const int cnt = seg_e - seg_s;
         if (seg_s >= p0 && seg_e <= p1) {   // the whole cluster lies in this range
-            if constexpr (EMA) finalize_ema<T, V>(p, rowbase + acck, lane, acc, wacc, cnt, WEIGHTED);
+            if constexpr (EMA) finalize_ema<T, V>(p, rowbase + acck, lane, acc, wacc, cnt, WEIGHTED, pre);
             else finalize_one<T, V>(p, rowbase + acck, lane, acc, wacc, cnt, WEIGHTED);
             return;
         }
@@ -729,7 +751,7 @@ __global__ void __launch_bounds__(fz_warps(32 * V * sizeof(T)) * 32, 1)
             for (int e = 0; e < V; ++e) tot[e] += __ldcg(q + e);
             wt += __ldcg(p.wslots + sl);
         }
-        if constexpr (EMA) finalize_ema<T, V>(p, rowbase + acck, lane, tot, wt, cnt, WEIGHTED);
+        if constexpr (EMA) finalize_ema<T, V>(p, rowbase + acck, lane, tot, wt, cnt, WEIGHTED, pre);
         else finalize_one<T, V>(p, rowbase + acck, lane, tot, wt, cnt, WEIGHTED);
     };
 
@@ -803,6 +825,7 @@ __global__ void __launch_bounds__(fz_warps(32 * V * sizeof(T)) * 32, 1)
                 acck = __shfl_sync(FULL, my_k, rr);
                 seg_s = __shfl_sync(FULL, my_s, rr);
                 seg_e = __shfl_sync(FULL, my_e, rr);
+                if constexpr (EMA) ema_prefetch<T, V>(p, rowbase + acck, lane, pre);
 #pragma unroll
                 for (int e = 0; e < V; ++e) acc[e] = 0.f;
                 wacc = 0.f;
