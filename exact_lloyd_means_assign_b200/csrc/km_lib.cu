@@ -1639,6 +1639,25 @@ km_status km_fit_host(const void *X_host, km_dtype dtype, const float *w_host, i
     cudaStream_t st = S(stream);
     const size_t xb = static_cast<size_t>(B * N * d) * dtype_size(dtype);
     const size_t cb = static_cast<size_t>(B * K * d) * 4;
+    // One iteration without labels: X is needed once, so it is streamed in 16 chunks (the
+    // out-of-core fit) and each chunk's assignment and accumulation overlap the next chunk's
+    // copy; the X staging area serves as that fit's workspace.
+    if (iters == 1 && !ids_host && xb >= (size_t{64} << 20)) {
+        const int64_t chunk = std::max<int64_t>(256, (ceil_div(N, 16) + 255) / 256 * 256);
+        const size_t need = km_stream_workspace_size(B, K, d, dtype, w_host != nullptr, chunk);
+        if (chunk < N && need > 0 && need <= xb) {
+            if (cudaMemcpyAsync(h.C, C_host, cb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+                return KM_ERR_CUDA;
+            km_status s = do_fit_stream(X_host, dtype, w_host, B, N, K, d, h.C, 1, chunk,
+                                        inertia_host ? h.inertia : nullptr, h.X, st);
+            if (s != KM_OK) return s;
+            if (cudaMemcpyAsync(C_host, h.C, cb, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+                (inertia_host && cudaMemcpyAsync(inertia_host, h.inertia, static_cast<size_t>(B) * 8,
+                                                 cudaMemcpyDeviceToHost, st) != cudaSuccess))
+                return KM_ERR_CUDA;
+            return cudaStreamSynchronize(st) == cudaSuccess ? KM_OK : KM_ERR_CUDA;
+        }
+    }
     if (cudaMemcpyAsync(h.X, X_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         (w_host && cudaMemcpyAsync(h.w, w_host, static_cast<size_t>(B * N) * 4,
                                    cudaMemcpyHostToDevice, st) != cudaSuccess) ||

@@ -198,11 +198,12 @@ km_status km_init_grid1d(const void *X, km_dtype dtype, int64_t B, int64_t N, in
  * kernel sorts every row once and stores the sorted values, indices and fp64 prefix sums of w,
  * w*x, w*x^2 in the workspace (32 bytes per point), then one kernel runs all iterations with a
  * warp per row; for 32 < K <= 64 one fused kernel per row keeps the row on chip (no workspace
- * needed). Small problems (K * d <= 4096, d <= 64, B * ceil(N / 256) <= 2048 CTAs that can all
+ * needed). Small problems (K * d <= 4096, d <= 64, B * ceil(N / 64) <= 2048 CTAs that can all
  * be resident, B * N * K * d <= 2^27, iters > 0) run the whole fit in one cooperative launch:
- * each CTA keeps 256 points in registers and assigns them with the same fp32 direct-form
- * arithmetic as the CUDA-core assignment, per-CTA partial sums are combined in CTA order after
- * a grid barrier whose waits are bounded like every other wait of the library. Everything else
+ * each CTA keeps 64 points in registers (four threads per point) and assigns them with the same
+ * fp32 direct-form arithmetic as the CUDA-core assignment; each CTA adds its per-cluster partial
+ * sums into the iteration's totals with atomics, and a grid barrier whose waits are bounded like
+ * every other wait of the library separates the iterations. Everything else
  * chains km_prep / km_assign / km_update on the stream. `ws` must hold
  * km_workspace_size(KM_OP_FIT, ...) bytes (else KM_ERR_WORKSPACE).
  */
@@ -216,6 +217,12 @@ km_status km_fit(const void *X, km_dtype dtype, const float *w, int64_t B, int64
  * when non-NULL, ids into ids_host[B,N] and the inertia history into inertia_host[iters,B],
  * then synchronises `stream`. Host buffers should be pinned for full PCIe bandwidth. The
  * workspace (device memory) is sized by km_workspace_size(KM_OP_FIT_HOST, ..., weighted, iters).
+ * With iters == 1, ids_host NULL and X of 64 MiB or more, X is needed only once: the call then
+ * streams X in 16 chunks of points (each a slice of every problem, as km_fit_stream does),
+ * with its buffers inside the X staging area, so the copy of one chunk overlaps the assignment
+ * and accumulation of the previous one. The labels are the same
+ * as km_fit's; the sums are accumulated chunk by chunk, so C and the inertia match km_fit's to
+ * fp32 (fp64 for the inertia) rounding, not bit for bit.
  */
 km_status km_fit_host(const void *X_host, km_dtype dtype, const float *w_host, int64_t B,
                       int64_t N, int64_t K, int64_t d, float *C_host, int iters, int32_t *ids_host,

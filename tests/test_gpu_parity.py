@@ -432,6 +432,28 @@ def test_fit_host_matches_device(cuda_device):
     assert (idsh.numpy() != to_np(ids)).mean() < 1e-3
 
 
+@pytest.mark.parametrize("dtype,N,weighted", [(torch.float16, 262144, False),
+                                               (torch.bfloat16, 270001, True)])
+def test_fit_host_single_iteration_streamed(dtype, N, weighted, cuda_device):
+    # X of 64 MiB or more, one iteration, no labels: km_fit_host streams X in 16 chunks (the last
+    # one ragged for N = 270001); the result matches the resident fit up to summation order
+    B, K, d = 1, 1024, 128
+    g = torch.Generator().manual_seed(11)
+    X = (torch.randn(B, N, d, generator=g) * 2).to(dtype)
+    C0 = X[:, torch.randperm(N, generator=g)[:K]].float().contiguous()
+    w = torch.rand(B, N, generator=g) + 0.5 if weighted else None
+    Xh, Ch = X.pin_memory(), C0.clone().pin_memory()
+    wh = w.pin_memory() if weighted else None
+    inh = torch.empty((1, B), dtype=torch.float64).pin_memory()
+    km.km_fit_host(Xh, Ch, 1, w_host=wh, inertia_host=inh)
+    Cd = C0.to(cuda_device)
+    _, _, ih, _ = km.km_fit(X.to(cuda_device), Cd, 1, w=w.to(cuda_device) if weighted else None,
+                            want_inertia=True)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(Ch, Cd.cpu(), rtol=1e-5, atol=1e-5)
+    np.testing.assert_allclose(inh.numpy(), to_np(ih), rtol=1e-9)
+
+
 STREAM_CASES = {
     # (dtype, B, N, K, d, chunk, weighted): ragged last chunk, several tiles per chunk
     "f16_tc": (torch.float16, 2, 5000, 300, 128, 1536, False),
