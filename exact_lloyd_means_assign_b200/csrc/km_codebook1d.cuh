@@ -27,67 +27,113 @@ constexpr int ENC_THREADS = 256;
 constexpr int ENC_VPT = 16;     // values per thread per block
 constexpr int ENC_KMAX = 256;   // 8-bit indices
 
-template <typename T>
+// Log2 of the search span: the smallest power of two above K (the count of sorted entries at or
+// below a value runs from 0 to K).
+__host__ __device__ constexpr int enc_logp(int K) {
+    int l = 0;
+    while ((1 << l) <= K) ++l;
+    return l;
+}
+
+// LOGP = enc_logp(K), fixed per instantiation so the binary search unrolls and a thread's values
+// are searched side by side. VEC: N is a multiple of 16 and X, codes are 16-byte aligned, so a
+// thread reads its 16 consecutive values with vector loads and writes their codes as one 16-byte
+// store; otherwise thread t takes values t, t + 256, ... of the block's range.
+template <typename T, int LOGP, bool VEC>
 __global__ void __launch_bounds__(ENC_THREADS)
     encode1d_kernel(const T *__restrict__ X, int64_t N, const float *__restrict__ C, int K,
                     uint8_t *__restrict__ codes) {
-    __shared__ float sv[2 * ENC_KMAX];   // rounded centroids, ascending by (value, index), then +inf
+    constexpr int P = 1 << LOGP;
+    __shared__ float cv[ENC_KMAX];       // the rounded centroids in index order
+    __shared__ float sv[P];              // the same ascending by (value, index), then NaN
     __shared__ int si[ENC_KMAX];         // their indices
+    __shared__ float4 br[ENC_KMAX + 1];  // per count lo of entries <= x: sorted entries lo-1, lo,
+    __shared__ int2 bi[ENC_KMAX + 1];    // lo-2, lo+1 (+-inf past the ends); indices of lo-1, lo
     const int b = blockIdx.y, tid = threadIdx.x;
+    const T *xb = X + static_cast<int64_t>(b) * N;
+    uint8_t *ob = codes + static_cast<int64_t>(b) * N;
+    const int64_t base = static_cast<int64_t>(blockIdx.x) * (ENC_THREADS * ENC_VPT);
+    // this thread's values are requested first, so their latency overlaps the codebook's setup
+    float x[ENC_VPT];
+    const int64_t i0 = base + static_cast<int64_t>(tid) * ENC_VPT;
+    const bool vin = VEC && i0 < N;   // the vector form's values are all in range or all out
+    if constexpr (VEC) {
+        constexpr int PER = 16 / sizeof(T);   // values per 16-byte load
+        uint4 raw[ENC_VPT / PER];
+#pragma unroll
+        for (int q = 0; q < ENC_VPT / PER; ++q)
+            raw[q] = vin ? __ldg(reinterpret_cast<const uint4 *>(xb + i0) + q) : make_uint4(0, 0, 0, 0);
+        const T *tv = reinterpret_cast<const T *>(raw);
+#pragma unroll
+        for (int v = 0; v < ENC_VPT; ++v) x[v] = Cvt<T>::to_f(tv[v]);
+    } else {
+#pragma unroll
+        for (int v = 0; v < ENC_VPT; ++v) {
+            const int64_t i = base + static_cast<int64_t>(v) * ENC_THREADS + tid;
+            x[v] = i < N ? Cvt<T>::to_f(xb[i]) : 0.f;
+        }
+    }
     const float *Cb = C + static_cast<int64_t>(b) * K;
-    int P = 1;   // the search runs over P > K entries, a power of two (so lo can reach K)
-    while (P <= K) P <<= 1;
-    for (int t = K + tid; t < P; t += ENC_THREADS) sv[t] = INFINITY;
+    if (tid < K) cv[tid] = round_through<T>(Cb[tid]);
+    // NaN padding: `pad <= x` is false for every x, so the count never runs past K
+    for (int t = K + tid; t < P; t += ENC_THREADS) sv[t] = __int_as_float(0x7fffffff);
+    __syncthreads();
     if (tid < K) {
-        const float v = round_through<T>(Cb[tid]);
+        const float v = cv[tid];
         int r = 0;
         for (int j = 0; j < K; ++j) {
-            const float u = round_through<T>(Cb[j]);
+            const float u = cv[j];
             r += (u < v) || (u == v && j < tid);
         }
         sv[r] = v;
         si[r] = tid;
     }
     __syncthreads();
-    const T *xb = X + static_cast<int64_t>(b) * N;
-    uint8_t *ob = codes + static_cast<int64_t>(b) * N;
-    const int64_t base = static_cast<int64_t>(blockIdx.x) * (ENC_THREADS * ENC_VPT);
-    // all of this thread's values are requested before any is encoded (one memory latency)
-    T xr[ENC_VPT];
-#pragma unroll
-    for (int v = 0; v < ENC_VPT; ++v) {
-        const int64_t i = base + static_cast<int64_t>(v) * ENC_THREADS + tid;
-        xr[v] = i < N ? xb[i] : Cvt<T>::from_f(0.f);
+    for (int lo = tid; lo <= K; lo += ENC_THREADS) {
+        br[lo] = make_float4(lo > 0 ? sv[lo - 1] : -INFINITY, lo < K ? sv[lo] : INFINITY,
+                             lo > 1 ? sv[lo - 2] : -INFINITY, lo + 1 < K ? sv[lo + 1] : INFINITY);
+        bi[lo] = make_int2(si[lo > 0 ? lo - 1 : 0], si[lo < K ? lo : K - 1]);
     }
+    __syncthreads();
+    uint32_t packed[ENC_VPT / 4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int v = 0; v < ENC_VPT; ++v) {
-        const int64_t i = base + static_cast<int64_t>(v) * ENC_THREADS + tid;
-        if (i >= N) break;
-        const float x = Cvt<T>::to_f(xr[v]);
-        int lo = 0;   // number of sorted entries <= x (branch-free, log2 P steps)
-        for (int step = P >> 1; step > 0; step >>= 1)
-            if (sv[lo + step - 1] <= x) lo += step;
-        const float tl = lo > 0 ? x - sv[lo - 1] : INFINITY;
-        const float tr = lo < K ? x - sv[lo] : INFINITY;
+        const float xv = x[v];
+        int lo = 0;   // number of sorted entries <= x
+#pragma unroll
+        for (int s = LOGP - 1; s >= 0; --s)
+            if (sv[lo + (1 << s) - 1] <= xv) lo += 1 << s;
+        const float4 e = br[lo];
+        const int2 ix = bi[lo];
+        // the nearest sits on one of the two entries bracketing x (an infinite side never wins)
+        const float tl = xv - e.x, tr = xv - e.y;
         const float dl = tl * tl, dr = tr * tr;
         const float best = fminf(dl, dr);
-        int idx = min(dl == best ? si[max(lo - 1, 0)] : K, dr == best ? si[min(lo, K - 1)] : K);
+        int idx = dr < dl ? ix.y : ix.x;
+        if (dr == dl) idx = min(ix.x, ix.y);
         // a third centroid can tie only with exactly the same rounded distance (rare)
-        float t2 = lo > 1 ? x - sv[lo - 2] : INFINITY;
-        float t3 = lo + 1 < K ? x - sv[lo + 1] : INFINITY;
+        const float t2 = xv - e.z, t3 = xv - e.w;
         if (t2 * t2 == best || t3 * t3 == best) {
             for (int q = lo - 2; q >= 0; --q) {   // distances grow leftwards
-                const float t = x - sv[q];
+                const float t = xv - sv[q];
                 if (t * t != best) break;
                 idx = min(idx, si[q]);
             }
             for (int q = lo + 1; q < K; ++q) {    // and rightwards
-                const float t = x - sv[q];
+                const float t = xv - sv[q];
                 if (t * t != best) break;
                 idx = min(idx, si[q]);
             }
         }
-        ob[i] = static_cast<uint8_t>(idx);
+        if constexpr (VEC) {
+            packed[v >> 2] |= static_cast<uint32_t>(idx & 0xff) << (8 * (v & 3));
+        } else {
+            const int64_t i = base + static_cast<int64_t>(v) * ENC_THREADS + tid;
+            if (i < N) ob[i] = static_cast<uint8_t>(idx);
+        }
+    }
+    if constexpr (VEC) {
+        if (vin) *reinterpret_cast<uint4 *>(ob + i0) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     }
 }
 

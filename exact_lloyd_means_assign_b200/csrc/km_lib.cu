@@ -1350,6 +1350,21 @@ inline bool emeans_fused_ok(km_dtype dt, const void *X, int64_t B, int64_t N, in
     return final_ok(dt, X, B, N, d);
 }
 
+template <typename T, int LOGP>
+void launch_encode1d(const void *X, int64_t N, const float *C, int K, uint8_t *codes, dim3 grid,
+                     bool vec, cudaStream_t st) {
+    using namespace km::cb;
+    const T *x = static_cast<const T *>(X);
+    if (vec) encode1d_kernel<T, LOGP, true><<<grid, ENC_THREADS, 0, st>>>(x, N, C, K, codes);
+    else encode1d_kernel<T, LOGP, false><<<grid, ENC_THREADS, 0, st>>>(x, N, C, K, codes);
+}
+
+template <typename T, int... L>
+void encode1d_by_logp(int logp, const void *X, int64_t N, const float *C, int K, uint8_t *codes,
+                      dim3 grid, bool vec, cudaStream_t st, std::integer_sequence<int, L...>) {
+    ((logp == L + 1 ? launch_encode1d<T, L + 1>(X, N, C, K, codes, grid, vec, st) : void()), ...);
+}
+
 }  // namespace
 
 // =================================================================== exported C ABI
@@ -1577,6 +1592,11 @@ km_status km_encode1d(const void *X, km_dtype dtype, int64_t B, int64_t N, const
         return KM_ERR_INVALID_ARG;
     cudaStream_t st = S(stream);
     const size_t esz = dtype_size(dtype);
+    const int k = static_cast<int>(K);
+    const int logp = enc_logp(k);   // 1 .. 9 for K = 1 .. 256
+    // the vector form: whole 16-value groups, every row starting on a 16-byte boundary
+    const bool vec = N % ENC_VPT == 0 && aligned(X, 16) && aligned(codes, 16);
+    using Seq = std::make_integer_sequence<int, 9>;
     for (int64_t b0 = 0; b0 < B; b0 += kMaxGridY) {   // rows in slices of the grid's y extent
         const int64_t nb = std::min<int64_t>(kMaxGridY, B - b0);
         const dim3 grid(static_cast<unsigned>(ceil_div(N, ENC_THREADS * ENC_VPT)), static_cast<unsigned>(nb));
@@ -1584,17 +1604,9 @@ km_status km_encode1d(const void *X, km_dtype dtype, int64_t B, int64_t N, const
         const float *Cs = C + b0 * K;
         uint8_t *out = codes + b0 * N;
         switch (dtype) {
-            case KM_F32:
-                encode1d_kernel<float><<<grid, ENC_THREADS, 0, st>>>(static_cast<const float *>(Xs), N,
-                                                                     Cs, static_cast<int>(K), out);
-                break;
-            case KM_F16:
-                encode1d_kernel<__half><<<grid, ENC_THREADS, 0, st>>>(static_cast<const __half *>(Xs), N,
-                                                                      Cs, static_cast<int>(K), out);
-                break;
-            default:
-                encode1d_kernel<__nv_bfloat16><<<grid, ENC_THREADS, 0, st>>>(
-                    static_cast<const __nv_bfloat16 *>(Xs), N, Cs, static_cast<int>(K), out);
+            case KM_F32: encode1d_by_logp<float>(logp, Xs, N, Cs, k, out, grid, vec, st, Seq{}); break;
+            case KM_F16: encode1d_by_logp<__half>(logp, Xs, N, Cs, k, out, grid, vec, st, Seq{}); break;
+            default: encode1d_by_logp<__nv_bfloat16>(logp, Xs, N, Cs, k, out, grid, vec, st, Seq{});
         }
         if (launch_status() != KM_OK) return KM_ERR_CUDA;
     }
