@@ -360,7 +360,10 @@ km_status km_split_dead(float *C, float *sizes, const float *u, float eps, int64
  * Weight Clustering ...": values stored as 8-bit indices of shared cluster values). Each value
  * X[b,i] becomes the index of its nearest centroid C[b,k] (centroids rounded to `dtype`, fp32
  * squared distance, lowest index on ties: the same decision as km_assign with d = 1), found by
- * binary search in the per-row sorted codebook.
+ * binary search in the per-row sorted codebook. Unlike the other calls, infinite values are
+ * defined here: every centroid is then at infinite distance, so the value gets index 0 (NaN
+ * values still get an unspecified index below K). Rows of N a multiple of 16 with X and codes
+ * 16-byte aligned are read and written with 16-byte vector accesses.
  *   X[B,N] in `dtype`, C[B,K] fp32 (any order), codes[B,N] uint8 out; all device memory.
  * K <= 256. Asynchronous on `stream`. Errors: KM_ERR_INVALID_ARG, KM_ERR_CUDA.
  */
