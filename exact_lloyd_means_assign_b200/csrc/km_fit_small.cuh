@@ -19,10 +19,11 @@
 //      clusters kept), so no second barrier is needed before the next assignment.
 // Three accumulators rotate: iteration t adds into A[t % 3], reads it after the barrier and
 // clears A[(t + 2) % 3], which every CTA finished reading before that barrier.
-// The barrier is a counter and a generation word in global memory; waits are bounded (the
-// library's wait limit, globaltimer), and a timeout sets the device error word and an abort
-// word that every CTA checks, so no CTA waits forever (km_debug_inject(2) makes CTA 0 skip its
-// first arrival so that a test can watch this happen).
+// The barrier is a counter and a generation word in global memory, ordered by acquire-release
+// operations rather than full fences; waits are bounded (the library's wait limit,
+// globaltimer), and a timeout sets the device error word and an abort word that every CTA
+// checks, so no CTA waits forever (km_debug_inject(2) makes CTA 0 skip its first arrival so
+// that a test can watch this happen).
 #pragma once
 
 #include "km_common.cuh"
@@ -47,24 +48,42 @@ struct Params {
     unsigned int *bar;        // [0] arrival count, [1] generation, [2] abort (zero at launch)
 };
 
+__device__ __forceinline__ unsigned int atom_add_acq_rel_gpu(unsigned int *p, unsigned int v) {
+    unsigned int old;
+    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(unsigned int *p, unsigned int v) {
+    asm volatile("st.release.gpu.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_relaxed_gpu(unsigned int *p, unsigned int v) {
+    asm volatile("st.relaxed.gpu.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Bounded grid barrier (all CTAs resident). Returns false once any CTA has given up.
+// Thread 0 of each CTA arrives with an acquire-release add (after the CTA barrier, so it
+// publishes the whole CTA's writes); the last to arrive resets the count and publishes the next
+// generation with a release store, which the others read with acquire loads.
 __device__ __forceinline__ bool grid_sync(unsigned int *bar, unsigned int nblocks, unsigned int &gen) {
     __shared__ int ok_s;
     __syncthreads();
     if (threadIdx.x == 0) {
         int ok = 1;
-        __threadfence();
         // test-only fault switch (off by default): CTA 0 never arrives at the first barrier
         const bool skip = gen == 0 && blockIdx.x == 0 && *reinterpret_cast<volatile int *>(&g_km_inject) == 2;
-        if (!skip && atomicAdd(bar, 1u) == nblocks - 1) {
-            atomicExch(bar, 0u);
-            __threadfence();
-            atomicExch(bar + 1, gen + 1);   // release the others
+        if (!skip && atom_add_acq_rel_gpu(bar, 1u) == nblocks - 1) {
+            st_relaxed_gpu(bar, 0u);          // ordered before the release below
+            st_release_gpu(bar + 1, gen + 1);   // release the others
         } else {
             const unsigned long long t0 = globaltimer_ns();
             const unsigned long long limit =
                 *reinterpret_cast<volatile unsigned long long *>(&g_km_wait_limit_ns);
-            while (*reinterpret_cast<volatile unsigned int *>(bar + 1) == gen) {
+            while (ld_acquire_gpu(bar + 1) == gen) {
                 if (*reinterpret_cast<volatile unsigned int *>(bar + 2)) { ok = 0; break; }
                 if (globaltimer_ns() - t0 > limit) {
                     record_dev_error(kDevErrTimeout);
@@ -72,10 +91,8 @@ __device__ __forceinline__ bool grid_sync(unsigned int *bar, unsigned int nblock
                     ok = 0;
                     break;
                 }
-                __nanosleep(32);
             }
         }
-        __threadfence();
         ok_s = ok && *reinterpret_cast<volatile unsigned int *>(bar + 2) == 0;
     }
     __syncthreads();
