@@ -37,6 +37,9 @@ def _separated(B, N, K, d, seed, far=0):
     ("f16", 2, 3000, 40, 24, True, 3),      # 17..32 coordinates; empty clusters
     ("bf16", 3, 700, 17, 64, True, 0),      # 33..64 coordinates, ragged last CTA
     ("f32", 2, 1000, 64, 2, True, 5),
+    ("f32", 4, 200, 8, 3, False, 0),        # one CTA per problem
+    ("f32", 1, 9000, 32, 16, False, 0),     # 141 CTAs
+    ("bf16", 2, 5000, 20, 40, True, 2),
 ])
 def test_small_fit_matches_oracle(dt, B, N, K, d, weighted, far, cuda_device):
     dtype = DT[dt]
