@@ -51,7 +51,7 @@ def test_single_rank_selftest_runs_in_process():
 def test_median_and_update_bytes():
     assert bench._median([3.0, 1.0, 2.0]) == 2.0
     assert bench._median([4.0, 1.0, 2.0, 3.0]) == 2.5
-    # the survey's algorithmic bytes of the headline update: X once + 4 passes over int32 ids
+    # the algorithmic bytes of the headline update: X once + 4 passes over int32 ids
     assert bench.UPDATE_BYTES == 32 * 65536 * 128 * 2 + 4 * 32 * 65536 * 4
 
 
