@@ -236,6 +236,8 @@ UPD_CASES = [
     ("f16", 1, 30000, 20000, 128),   # K above the 16384 shared-memory bins: the two-launch sort
     ("f16", 2, 20000, 4096, 128),    # the largest K whose scatter tiles are sorted in shared memory
     ("bf16", 1, 20000, 4097, 64),    # one above: labels ranked straight into perm
+    ("f16", 1, 40000, 16384, 128),   # the largest K whose counts are scanned in shared memory
+    ("f16", 1, 40000, 16385, 64),    # one above: the separate scan launch
 ]
 
 
