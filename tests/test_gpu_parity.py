@@ -528,3 +528,24 @@ def test_fit_k_greater_than_n_keeps_empty(cuda_device):
     ids1, _, _, _ = oracle.assign(oracle.as_f64(X.cpu()), oracle.round_to_dtype(ch[1].cpu(), torch.float16))
     never = np.setdiff1d(never, np.unique(ids1[0]))
     np.testing.assert_array_equal(to_np(C)[0, never], to_np(C0)[0, never])
+
+
+def test_more_problems_than_the_grid_y_limit(cuda_device):
+    # 65600 problems: the launches that put problems on the grid's y axis (65535 at most) run
+    # in slices; every problem must come out as if it were alone
+    B, N, K, d = 65600, 32, 4, 32
+    X, C = mixture(B, N, d, K, torch.float16, cuda_device, seed=5)
+    Cx, cn = km.km_prep(C, torch.float16)
+    ids, _, _ = km.km_assign(X, Cx, cn)
+    C_new, counts, _ = km.km_update(X, ids, C)
+    torch.cuda.synchronize()
+    check_assign(X, C, ids)
+    check_update(X, ids, C, C_new, counts)
+    # 1-D encoding of as many rows
+    vals = X[:, :, 0].contiguous()
+    cents = C[:, :, 0].contiguous()
+    codes = km.km_encode1d(vals, cents)
+    torch.cuda.synchronize()
+    from oracle import codebook1d
+    ref, d1, d2 = codebook1d.encode1d(oracle.as_f64(vals.cpu()), oracle.as_f64(cents.cpu()), torch.float16)
+    assert not ((to_np(codes) != ref) & ~oracle.near_tie(d1, d2)).any()
