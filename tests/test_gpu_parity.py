@@ -530,10 +530,11 @@ def test_fit_k_greater_than_n_keeps_empty(cuda_device):
     np.testing.assert_array_equal(to_np(C)[0, never], to_np(C0)[0, never])
 
 
-def test_more_problems_than_the_grid_y_limit(cuda_device):
+@pytest.mark.parametrize("d", [32, 64])   # 64-byte rows: the sums-array update; 128: the fused one
+def test_more_problems_than_the_grid_y_limit(d, cuda_device):
     # 65600 problems: the launches that put problems on the grid's y axis (65535 at most) run
     # in slices; every problem must come out as if it were alone
-    B, N, K, d = 65600, 32, 4, 32
+    B, N, K = 65600, 32, 4
     X, C = mixture(B, N, d, K, torch.float16, cuda_device, seed=5)
     Cx, cn = km.km_prep(C, torch.float16)
     ids, _, _ = km.km_assign(X, Cx, cn)
