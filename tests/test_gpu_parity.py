@@ -64,6 +64,7 @@ TC_CASES = [
     ("f16", 1, 129, 1, 128),
     ("f16", 2, 100, 300, 24),
     ("bf16", 5, 1, 7, 8),
+    ("bf16", 1, 600, 40000, 64),     # 157 centroid tiles streamed through the ring
 ]
 SIMT_CASES = [
     ("f32", 1, 4096, 32, 16),
