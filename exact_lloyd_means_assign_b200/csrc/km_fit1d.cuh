@@ -469,7 +469,10 @@ __global__ void __launch_bounds__(THREADS, 4)
     }
 }
 
-template <typename T>
+// KT: a power of two >= K, fixed per instantiation, so every lane keeps the rounded centroids in
+// registers for the whole iteration (entries K .. KT-1 hold NaN, which never compares below a
+// distance) and a probe's scan over them is unrolled with no memory access.
+template <typename T, int KT>
 __global__ void __launch_bounds__(ITER_WARPS * 32)
     fit1d_iter_kernel(const float *__restrict__ xs, const int32_t *__restrict__ is,
                       const double *__restrict__ P0, const double *__restrict__ P1,
@@ -510,6 +513,12 @@ __global__ void __launch_bounds__(ITER_WARPS * 32)
             orderw[r] = lane;
         }
         __syncwarp();
+        float creg[KT];
+#pragma unroll
+        for (int k = 0; k < KT; ++k) {
+            const float v = __shfl_sync(FULL, cxk, k);
+            creg[k] = k < K ? v : __int_as_float(0x7fffffff);
+        }
         // boundary q = lane: first sorted position whose nearest centroid ranks above q
         int lo = 0, len = N;
         for (int st = 0; st < steps; ++st) {
@@ -518,8 +527,9 @@ __global__ void __launch_bounds__(ITER_WARPS * 32)
             const float x = len > 0 ? xr[mid] : 0.f;
             float best = INFINITY;
             int bi = 0;
-            for (int k = 0; k < K; ++k) {
-                const float dx = x - cxw[k];
+#pragma unroll
+            for (int k = 0; k < KT; ++k) {   // the first strict minimum: the lowest index on ties
+                const float dx = x - creg[k];
                 const float dd = dx * dx;
                 if (dd < best) {
                     best = dd;

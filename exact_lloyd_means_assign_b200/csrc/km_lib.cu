@@ -924,9 +924,16 @@ km_status run_fit1d(const void *X, const float *w, int64_t B, int64_t N, int64_t
             static_cast<const T *>(X), w, static_cast<int>(N), NR, g.xs, g.is, g.P0, g.P1,
             inertia_hist ? g.P2 : nullptr);
         if (launch_status() != KM_OK) return KM_ERR_CUDA;
-        fit1d_iter_kernel<T><<<static_cast<unsigned>(ceil_div(B, ITER_WARPS)), ITER_WARPS * 32, 0, st>>>(
-            g.xs, g.is, g.P0, g.P1, inertia_hist ? g.P2 : nullptr, static_cast<int>(B), static_cast<int>(N), static_cast<int>(K),
-            iters, C, ids, inertia_hist, C_hist);
+        auto iter = [&](auto kt) {
+            fit1d_iter_kernel<T, decltype(kt)::value><<<static_cast<unsigned>(ceil_div(B, ITER_WARPS)),
+                                                       ITER_WARPS * 32, 0, st>>>(
+                g.xs, g.is, g.P0, g.P1, inertia_hist ? g.P2 : nullptr, static_cast<int>(B),
+                static_cast<int>(N), static_cast<int>(K), iters, C, ids, inertia_hist, C_hist);
+        };
+        if (K <= 4) iter(std::integral_constant<int, 4>{});
+        else if (K <= 8) iter(std::integral_constant<int, 8>{});
+        else if (K <= 16) iter(std::integral_constant<int, 16>{});
+        else iter(std::integral_constant<int, 32>{});
         return launch_status();
     }
     const size_t smem = static_cast<size_t>(NP) * 12;
