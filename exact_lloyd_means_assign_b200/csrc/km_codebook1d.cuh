@@ -142,34 +142,42 @@ constexpr int PP_PER = 16;      // points per thread: rows of up to PP_THREADS *
 constexpr int PP_NMAX = PP_THREADS * PP_PER;
 
 // One block per row; thread t owns the contiguous points [t * per, t * per + per), so a block scan
-// of the per-thread masses gives running sums in point order.
-template <typename T>
-__global__ void __launch_bounds__(PP_THREADS)
+// of the per-thread masses gives running sums in point order. PER >= per bounds the thread's
+// arrays: rows of up to 4096 values take PER = 8, which leaves room for two blocks per SM.
+template <typename T, int PER>
+__global__ void __launch_bounds__(PP_THREADS, PER <= 8 ? 2 : 1)
     kmeanspp1d_kernel(const T *__restrict__ X, const float *__restrict__ w, int N, int K,
                       const float *__restrict__ u, float *__restrict__ C,
                       int32_t *__restrict__ chosen) {
     constexpr int NW = PP_THREADS / 32;
     __shared__ double wtot[NW];
-    __shared__ int pick, last_mass;
+    __shared__ int last_mass;
+    // the chosen point as (index << 32) | its value's bits, all ones while none: the lowest
+    // claimant wins, and the index and value always come from the same thread
+    __shared__ unsigned long long pick;
     const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int per = (N + PP_THREADS - 1) / PP_THREADS;
     const int p0 = min(N, tid * per);
     const int np = min(N, p0 + per) - p0;
     const int64_t rb = static_cast<int64_t>(b) * N;
-    float xv[PP_PER], wv[PP_PER];
-    double d2[PP_PER];
+    float xv[PER], wv[PER];
+    double d2[PER];
 #pragma unroll
-    for (int e = 0; e < PP_PER; ++e) {
+    for (int e = 0; e < PER; ++e) {
         const bool in = e < np;
         xv[e] = in ? Cvt<T>::to_f(X[rb + p0 + e]) : 0.f;
         wv[e] = in ? (w ? w[rb + p0 + e] : 1.f) : 0.f;
         d2[e] = 1.0;   // the first draw is proportional to the weights alone
     }
+    const float *ub = u + static_cast<int64_t>(b) * K;
+    float u_next = ub[0];   // each draw's uniform is requested one draw ahead
     for (int k = 0; k < K; ++k) {
+        const float uk = u_next;
+        if (k + 1 < K) u_next = ub[k + 1];
         double loc = 0.0;
         int mylast = -1;   // this thread's last point with mass
 #pragma unroll
-        for (int e = 0; e < PP_PER; ++e) {
+        for (int e = 0; e < PER; ++e) {
             const double m = static_cast<double>(wv[e]) * d2[e];
             loc += m;
             if (e < np && m > 0.0) mylast = p0 + e;
@@ -182,7 +190,7 @@ __global__ void __launch_bounds__(PP_THREADS)
         }
         if (lane == 31) wtot[warp] = inc;
         if (tid == 0) {
-            pick = -1;
+            pick = ~0ull;
             last_mass = -1;
         }
         __syncthreads();
@@ -193,15 +201,15 @@ __global__ void __launch_bounds__(PP_THREADS)
             total += wtot[v];
         }
         if (total > 0.0) {
-            const double target = static_cast<double>(u[static_cast<int64_t>(b) * K + k]) * total;
+            const double target = static_cast<double>(uk) * total;
             double run = off + inc - loc;
             if (run <= target && run + loc > target) {
 #pragma unroll
-                for (int e = 0; e < PP_PER; ++e) {
+                for (int e = 0; e < PER; ++e) {
                     const double m = static_cast<double>(wv[e]) * d2[e];
                     run += m;
                     if (e < np && m > 0.0 && run > target) {
-                        pick = p0 + e;
+                        atomicMin(&pick, (static_cast<unsigned long long>(p0 + e) << 32) | __float_as_uint(xv[e]));
                         break;
                     }
                 }
@@ -209,16 +217,20 @@ __global__ void __launch_bounds__(PP_THREADS)
         }
         __syncthreads();
         // no mass left: point 0; rounding left the target at the total: the last point with mass
-        if (tid == 0 && pick < 0) pick = last_mass >= 0 ? last_mass : 0;
+        if (tid == 0 && pick == ~0ull) {
+            const int f = last_mass >= 0 ? last_mass : 0;
+            pick = (static_cast<unsigned long long>(f) << 32) | __float_as_uint(Cvt<T>::to_f(X[rb + f]));
+        }
         __syncthreads();
-        const int i = pick;
-        const float c = Cvt<T>::to_f(X[rb + i]);
+        const unsigned long long pv = pick;
+        const int i = static_cast<int>(pv >> 32);
+        const float c = __uint_as_float(static_cast<uint32_t>(pv));
         if (tid == 0) {
             C[static_cast<int64_t>(b) * K + k] = c;
             if (chosen) chosen[static_cast<int64_t>(b) * K + k] = i;
         }
 #pragma unroll
-        for (int e = 0; e < PP_PER; ++e) {
+        for (int e = 0; e < PER; ++e) {
             const double t = static_cast<double>(xv[e]) - static_cast<double>(c);
             const double dd = t * t;
             d2[e] = (k == 0) ? dd : fmin(d2[e], dd);

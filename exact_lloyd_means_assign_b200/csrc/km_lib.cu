@@ -1353,6 +1353,8 @@ km_status run_emeans_fused(const void *X, km_dtype dt, const float *w, int64_t B
     return KM_OK;
 }
 
+template <typename T> struct TypeTag { using type = T; };
+
 inline bool emeans_fused_ok(km_dtype dt, const void *X, int64_t B, int64_t N, int64_t d) {
     return final_ok(dt, X, B, N, d);
 }
@@ -1631,16 +1633,25 @@ km_status km_init_kmeanspp1d(const void *X, km_dtype dtype, const float *w, int6
     cudaStream_t st = S(stream);
     const unsigned grid = static_cast<unsigned>(B);
     const int n = static_cast<int>(N), k = static_cast<int>(K);
+    // rows of up to 4096 values: 8 points per thread (two blocks per SM), else 16
+    auto run = [&](auto tag, auto per) {
+        using T = typename decltype(tag)::type;
+        kmeanspp1d_kernel<T, decltype(per)::value><<<grid, PP_THREADS, 0, st>>>(
+            static_cast<const T *>(X), w, n, k, u, C, chosen);
+    };
+    const bool small = N <= PP_THREADS * 8;
     switch (dtype) {
         case KM_F32:
-            kmeanspp1d_kernel<float><<<grid, PP_THREADS, 0, st>>>(static_cast<const float *>(X), w, n, k, u, C, chosen);
+            if (small) run(TypeTag<float>{}, std::integral_constant<int, 8>{});
+            else run(TypeTag<float>{}, std::integral_constant<int, PP_PER>{});
             break;
         case KM_F16:
-            kmeanspp1d_kernel<__half><<<grid, PP_THREADS, 0, st>>>(static_cast<const __half *>(X), w, n, k, u, C, chosen);
+            if (small) run(TypeTag<__half>{}, std::integral_constant<int, 8>{});
+            else run(TypeTag<__half>{}, std::integral_constant<int, PP_PER>{});
             break;
         default:
-            kmeanspp1d_kernel<__nv_bfloat16><<<grid, PP_THREADS, 0, st>>>(
-                static_cast<const __nv_bfloat16 *>(X), w, n, k, u, C, chosen);
+            if (small) run(TypeTag<__nv_bfloat16>{}, std::integral_constant<int, 8>{});
+            else run(TypeTag<__nv_bfloat16>{}, std::integral_constant<int, PP_PER>{});
     }
     return launch_status();
 }
