@@ -195,11 +195,16 @@ __global__ void __launch_bounds__(PP_THREADS, PER <= 8 ? 2 : 1)
         }
         __syncthreads();
         if (mylast >= 0) atomicMax(&last_mass, mylast);
-        double total = 0.0, off = 0.0;
-        for (int v = 0; v < NW; ++v) {
-            if (v < warp) off += wtot[v];
-            total += wtot[v];
+        // the warps' totals scanned across the lanes of every warp: this warp's offset and the row's total
+        double ws = lane < NW ? wtot[lane] : 0.0;
+#pragma unroll
+        for (int o = 1; o < NW; o <<= 1) {
+            const double t = __shfl_up_sync(0xffffffffu, ws, o);
+            if (lane >= o) ws += t;
         }
+        const double total = __shfl_sync(0xffffffffu, ws, NW - 1);
+        const double wprev = __shfl_sync(0xffffffffu, ws, warp > 0 ? warp - 1 : 0);
+        const double off = warp > 0 ? wprev : 0.0;
         if (total > 0.0) {
             const double target = static_cast<double>(uk) * total;
             double run = off + inc - loc;
