@@ -704,11 +704,12 @@ inline bool final_ok(km_dtype dt, const void *X, int64_t B, int64_t N, int64_t d
 
 // Ranges of sorted positions for the fused reduce: one CTA per SM of `nw` warps, every warp one
 // range of one batch element (ranges need not be whole chunks of 32 positions, so every warp
-// gets one). Returns (range, ranges per batch element).
+// gets one), but no range shorter than one chunk: below that a warp's fixed costs outweigh its
+// rows. Returns (range, ranges per batch element).
 inline void final_ranges(int64_t B, int64_t N, int nw, int64_t &range, int64_t &rpb) {
     const int64_t total = static_cast<int64_t>(std::min(num_sms(), static_cast<int>(kFinalWarpsMax / nw))) * nw;
     const int64_t rpb0 = std::max<int64_t>(1, total / B);
-    range = std::max<int64_t>(64, ceil_div(N, rpb0));
+    range = std::max<int64_t>(32, ceil_div(N, rpb0));
     rpb = ceil_div(N, range);   // <= rpb0 < final_rpb_max(B)
 }
 
