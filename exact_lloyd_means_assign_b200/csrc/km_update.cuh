@@ -1005,6 +1005,29 @@ __device__ __forceinline__ int block_exscan(int *a, int K, int *wtot) {
     return carry;
 }
 
+// Each cluster present in a scatter tile gets its slot range: h[k] <- offs[k] + (old fill[k])
+// - base[k] (base null: 0), with fill[k] += h[k]. A thread's clusters are taken eight at a time
+// so that their atomics are in flight together instead of one round trip after another.
+__device__ __forceinline__ void reserve_slots(int *h, const int *offs, const int *base,
+                                              int32_t *__restrict__ fillb, int K, int tid) {
+    constexpr int RB = 8;
+    for (int k0 = tid; k0 < K; k0 += RB * TILE_THREADS) {
+        int hv[RB], r[RB];
+#pragma unroll
+        for (int u = 0; u < RB; ++u) {
+            const int k = k0 + u * TILE_THREADS;
+            hv[u] = k < K ? h[k] : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < RB; ++u) r[u] = hv[u] ? atomicAdd(fillb + k0 + u * TILE_THREADS, hv[u]) : 0;
+#pragma unroll
+        for (int u = 0; u < RB; ++u) {
+            const int k = k0 + u * TILE_THREADS;
+            if (hv[u]) h[k] = offs[k] + r[u] - (base ? base[k] : 0);
+        }
+    }
+}
+
 // The counting-sort scatter with the scan folded in (K <= SMEM_K_MAX; tile <= SCATTER_PPT *
 // TILE_THREADS, each thread keeping its points' labels in registers so the tile's histogram and
 // ranking issue all their shared-memory atomics back to back). With K <= SCATTER_SORT_K_MAX the
@@ -1108,8 +1131,7 @@ __global__ void __launch_bounds__(TILE_THREADS)
         __syncthreads();
         const int nvalid = block_exscan(lofs, K, wtot);
         // each cluster's slot range, kept as (global slot - tile-local position)
-        for (int k = tid; k < K; k += TILE_THREADS)
-            if (h[k]) h[k] = offs[k] + atomicAdd(&fill[kb + k], h[k]) - lofs[k];
+        reserve_slots(h, offs, lofs, fill + kb, K, tid);
         __syncthreads();
 #pragma unroll
         for (int m = 0; m < SCATTER_PPT; ++m)
@@ -1123,8 +1145,7 @@ __global__ void __launch_bounds__(TILE_THREADS)
         return;
     }
     // reserve each cluster of the tile a slot range, then rank the points into it
-    for (int k = tid; k < K; k += TILE_THREADS)
-        if (h[k]) h[k] = offs[k] + atomicAdd(&fill[kb + k], h[k]);
+    reserve_slots(h, offs, nullptr, fill + kb, K, tid);
     __syncthreads();
     int pos[SCATTER_PPT];
 #pragma unroll
