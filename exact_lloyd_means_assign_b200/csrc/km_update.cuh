@@ -1083,22 +1083,27 @@ __global__ void __launch_bounds__(TILE_THREADS)
     for (int m = 0; m < SCATTER_PPT; ++m)
         if (static_cast<unsigned>(lab[m]) < static_cast<unsigned>(K)) atomicAdd(&h[lab[m]], 1);
     __syncthreads();
-    // this problem's per-cluster work, split over its tiles
-    if (blockIdx.x == 0) {
-        for (int k = tid; k <= K; k += TILE_THREADS) offsets[static_cast<int64_t>(b) * (K + 1) + k] = offs[k];
-        // the segment holding the first position of each range of the reduction that follows
-        for (int r = tid; r < rpb; r += TILE_THREADS) {
-            const int p0 = r * range;
-            int lo = 0, hi = K - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (offs[mid] <= p0) lo = mid; else hi = mid - 1;
-            }
-            rseg[static_cast<int64_t>(b) * rpb + r] = lo;
-        }
-    }
+    // this problem's offsets and range-start table: every tile holds the whole scan, so with many
+    // clusters (the unsorted form) the tiles share the writing, else tile 0 does it alone
     const int kb0 = static_cast<int>(static_cast<int64_t>(K) * blockIdx.x / gridDim.x);
     const int kb1 = static_cast<int>(static_cast<int64_t>(K) * (blockIdx.x + 1) / gridDim.x);
+    const bool share = !sorted_form;
+    const int ok0 = share ? kb0 : (blockIdx.x == 0 ? 0 : K), ok1 = share ? kb1 : K;
+    for (int k = ok0 + tid; k < ok1; k += TILE_THREADS) offsets[static_cast<int64_t>(b) * (K + 1) + k] = offs[k];
+    if (blockIdx.x == (share ? gridDim.x - 1 : 0) && tid == 0) offsets[static_cast<int64_t>(b) * (K + 1) + K] = offs[K];
+    // the segment holding the first position of each range of the reduction that follows
+    const int rb0 = share ? static_cast<int>(static_cast<int64_t>(rpb) * blockIdx.x / gridDim.x)
+                          : (blockIdx.x == 0 ? 0 : rpb);
+    const int rb1 = share ? static_cast<int>(static_cast<int64_t>(rpb) * (blockIdx.x + 1) / gridDim.x) : rpb;
+    for (int r = rb0 + tid; r < rb1; r += TILE_THREADS) {
+        const int p0 = r * range;
+        int lo = 0, hi = K - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (offs[mid] <= p0) lo = mid; else hi = mid - 1;
+        }
+        rseg[static_cast<int64_t>(b) * rpb + r] = lo;
+    }
     for (int k = kb0 + tid; k < kb1; k += TILE_THREADS) {
         arrive[kb + k] = 0;
         if (Nc && offs[k + 1] == offs[k]) Nc[kb + k] *= 1.f - alpha;
