@@ -332,6 +332,8 @@ def test_fit1d_weighted_rows_per_iteration(K, cuda_device):
     ("bf16", 1000, 5, False),
     ("f16", 8192, 1, True),     # the largest row; one cluster
     ("f16", 700, 48, True),     # K > 32: the fused one-CTA-per-row form
+    ("f16", 2000, 20, True),    # 12 unused centroid registers of the 32-wide form
+    ("bf16", 1500, 12, False),  # 4 unused of the 16-wide form
 ])
 def test_fit1d_shapes_per_iteration(dt, N, K, weighted, cuda_device):
     g = torch.Generator().manual_seed(N + K)
